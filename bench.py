@@ -1,0 +1,428 @@
+"""Benchmark of the BlockFFN chunk-union layer forward at one n=32 verification chunk.
+
+Workload (one step = one layer call on one chunk): n = 32 tokens, d_h = 2048,
+E = 64 experts, d_e = 128, bf16, injected gates from a per-expert Markov chain
+(off->on 0.019, on->off 0.076: about 80 % token-level and 70 % 8-token
+chunk-level sparsity), active gate values |N(0,1)|, x ~ N(0,1), weights
+~ N(0, 1/fan_in).  Synthetic data (no trained model exists here).
+
+Device timing: R = 8 copies of (W_in, W_out, x, gates) rotate step by step, so
+the 512 MiB of weights exceed the 126 MB L2 and every step streams its union
+experts from HBM.  The K timed steps run as CUDA-graph replays on one stream,
+bracketed by a barrier and a device synchronize, with CUDA events; per-step
+events around each launch give the kernel's own time for the roofline.
+
+The JSON line also carries: the end-to-end number through the public API with
+host buffers (x and gates copied in from pinned memory, y copied out, every
+step), the same-size dense FFN on the GPU (torch bf16 matmuls) for context,
+the HBM roofline fraction on union-expert bytes, the fp64 CPU oracle timed on a
+bounded sample (rank 0, one GPU), and the SM clocks sampled during the run.
+
+``--impl reference`` times the fp64 CPU oracle alone on the same workload and
+metric (there is no runnable upstream implementation).
+Multi-GPU (torchrun): independent replicas, one per GPU, no collective on the
+data path (the layer does not shard); weak scaling, max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "tokens/s per BlockFFN layer at n=32 chunk"
+UNIT = "tokens/s"
+R_COPIES = 8
+L2_BYTES = 126 * 1024 * 1024
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the forward kernel,
+# from the ncu capture summarised in profiles/ (None until captured for the
+# current kernel).
+TRAFFIC_BYTES_PER_LAUNCH = None
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def union_bytes(w: wl.Workload) -> int:
+    """Algorithmic bytes of one call: every union expert's W_in_e and W_out_e once,
+    plus x, y (bf16) and the gates (fp32)."""
+    active = np.any(w.gates != 0, axis=0)
+    U = int(np.sum(active))
+    return U * 2 * w.d_h * w.d_e * 2 + 2 * w.T * w.d_h * 2 + w.T * w.E * 4
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=None)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    """The fp64 oracle (dense definition) on whole chunks of the workload, timed on
+    this host's cores for about ``budget_s`` seconds."""
+    import oracle
+    w = wl.chunk32()
+    x, g, Wi, Wo = (np.asarray(a, np.float64) for a in (w.x, w.gates, w.W_in, w.W_out))
+    oracle.forward_dense(x[:1], g[:1], Wi, Wo)  # build + warm
+    t0 = time.perf_counter()
+    tokens = 0
+    calls = 0
+    while True:
+        oracle.forward_dense(x, g, Wi, Wo)
+        tokens += w.T
+        calls += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{calls} dense fp64 oracle calls on the 32-token chunk "
+                      f"({w.T * calls} tokens, {dt:.1f} s)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    cb = cpu_baseline(budget_s=max(2.0, min(60.0, 1.0 * (args.steps + args.warmup) / 100)))
+    line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * 32 / cb["value"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": "chunk32: n=32, d_h=2048, E=64, d_e=128, Markov(0.019, 0.076)"
+                                   " gates; fp64 dense CPU oracle"},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    import chunk_sparse_moe_b200 as bffn
+
+    dev = torch.device("cuda", local)
+    dt = torch.bfloat16
+    base = wl.chunk32(seed=0)
+    copies = [base] + [wl.chunk32(seed=0, weights=(base.W_in, base.W_out), x_seed=k)
+                       for k in range(1, R_COPIES)]
+    W_in0 = torch.from_numpy(base.W_in).to(dev, dt)
+    W_out0 = torch.from_numpy(base.W_out).to(dev, dt)
+    bufs = []
+    for k, w in enumerate(copies):
+        bufs.append({
+            "x": torch.from_numpy(w.x).to(dev, dt),
+            "g": torch.from_numpy(w.gates).to(dev, torch.float32),
+            "W_in": W_in0 if k == 0 else W_in0.clone(),
+            "W_out": W_out0 if k == 0 else W_out0.clone(),
+            "y": torch.empty((w.T, w.d_h), dtype=dt, device=dev),
+        })
+    T, n, d_h, E, d_e = base.T, base.n, base.d_h, base.E, base.d_e
+    ws = bffn.Workspace.for_shapes(T, d_h, E, d_e, n, dt, False, dev)
+    alg_bytes = [union_bytes(w) for w in copies]
+    resident = sum(b["W_in"].numel() * 2 + b["W_out"].numel() * 2 for b in bufs)
+    assert resident > 2 * L2_BYTES
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(k):
+        b = bufs[k % R_COPIES]
+        bffn.forward(b["x"], b["W_in"], b["W_out"], n, gates=b["g"], y=b["y"], workspace=ws)
+
+    # correctness gate before timing: one call of every copy, finite output
+    with torch.cuda.stream(stream):
+        for k in range(R_COPIES):
+            step(k)
+    stream.synchronize()
+    st = bffn.device_status(ws)
+    if st[0] != 0:
+        raise SystemExit(f"device status {st} after warm-up")
+
+    # CUDA graphs of R steps (one per copy) and of the remainder
+    def capture(count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for k in range(count):
+                step(k)
+        return g
+
+    use_graph = not args.no_graph
+    graph_err = None
+    if use_graph:
+        try:
+            g_full = capture(R_COPIES)
+            rem = args.steps % R_COPIES
+            g_rem = capture(rem) if rem else None
+        except Exception as e:  # report and time eagerly
+            use_graph, graph_err = False, repr(e)
+            torch.cuda.synchronize()
+
+    def run_steps(count):
+        if use_graph:
+            for _ in range(count // R_COPIES):
+                g_full.replay()
+            if count % R_COPIES:
+                if count % R_COPIES == args.steps % R_COPIES and g_rem is not None:
+                    g_rem.replay()
+                else:
+                    for k in range(count % R_COPIES):
+                        step(k)
+        else:
+            for k in range(count):
+                step(k)
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    stream.synchronize()
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        run_steps(args.steps)
+        ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    clock_info = clocks.stop()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    st = bffn.device_status(ws)
+    if st[0] != 0:
+        raise SystemExit(f"device status {st} after the timed run")
+
+    # kernel-only time for the roofline: per-step events around single launches
+    # (a GPU-side sleep first, so every launch is queued before the GPU reaches it
+    # and the events see device time, not host launch gaps)
+    with torch.cuda.stream(stream):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(4 * R_COPIES)]
+        torch.cuda._sleep(100_000_000)
+        for k, (a, b) in enumerate(evs):
+            a.record(stream)
+            step(k)
+            b.record(stream)
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in evs]
+    kernel_ms = statistics.median(per)
+    mean_bytes = sum(alg_bytes) / len(alg_bytes)
+    hbm_peak, peak_kind = peaks()
+    achieved_gbs = mean_bytes / (kernel_ms * 1e-3) / 1e9
+    step_gbs = mean_bytes / (elapsed_ms / args.steps * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    x_h = [torch.from_numpy(w.x).to(dt).pin_memory() for w in copies]
+    g_h = [torch.from_numpy(w.gates).pin_memory() for w in copies]
+    y_h = [torch.empty((T, d_h), dtype=dt).pin_memory() for _ in copies]
+    e2e_steps = min(args.e2e_steps, args.steps)
+
+    def e2e_step(k):
+        b = bufs[k % R_COPIES]
+        b["x"].copy_(x_h[k % R_COPIES], non_blocking=True)
+        b["g"].copy_(g_h[k % R_COPIES], non_blocking=True)
+        bffn.forward(b["x"], b["W_in"], b["W_out"], n, gates=b["g"], y=b["y"], workspace=ws)
+        y_h[k % R_COPIES].copy_(b["y"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for k in range(max(3, args.warmup // 10)):
+            e2e_step(k)
+    stream.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for k in range(e2e_steps):
+            e2e_step(k)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = T * d_h * 2 + T * E * 4
+    d2h = T * d_h * 2
+
+    # same-size dense FFN on the GPU (torch bf16 matmuls), context only
+    W_in_cat = [b["W_in"].reshape(E * d_e, d_h) for b in bufs]
+    W_out_cat = [b["W_out"].permute(1, 0, 2).reshape(d_h, E * d_e) for b in bufs]
+    W_out_cat = [w.contiguous() for w in W_out_cat]
+
+    def dense(k):
+        b = bufs[k % R_COPIES]
+        h = torch.nn.functional.silu(b["x"] @ W_in_cat[k % R_COPIES].t())
+        return h @ W_out_cat[k % R_COPIES].t()
+
+    with torch.cuda.stream(stream):
+        for k in range(2 * R_COPIES):
+            dense(k)
+        dd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(4 * R_COPIES)]
+        torch.cuda._sleep(100_000_000)
+        for k, (a, b) in enumerate(dd):
+            a.record(stream)
+            dense(k)
+            b.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = statistics.median([a.elapsed_time(b) for a, b in dd])
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline()
+
+    if rank == 0:
+        value = world * T * args.steps / (elapsed_ms * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random-init weights, Markov gate masks)",
+            "config": {
+                "workload": "chunk32: one n=32 verification chunk, d_h=2048, E=64, d_e=128, "
+                            "bf16, injected gates Markov(0.019, 0.076), |N(0,1)| values",
+                "parallelism": f"replicas x{world} (no collective)",
+                "l2": f"{R_COPIES} rotating copies of weights/x/gates "
+                      f"({resident / 2**20:.0f} MiB > 126 MB L2)",
+                "launch": "CUDA graph replays" if use_graph else "eager",
+                "mean_union_experts": float(np.mean([np.sum(np.any(w.gates != 0, axis=0))
+                                                     for w in copies])),
+            },
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": achieved_gbs / hbm_peak,
+                         "traffic": TRAFFIC_BYTES_PER_LAUNCH,
+                         "peak_kind": peak_kind,
+                         "kernel": "union_expert_forward_tc",
+                         "kernel_us": kernel_ms * 1e3,
+                         "algorithmic_bytes_per_launch": mean_bytes,
+                         "step_gbs": step_gbs,
+                         "frac_of_8tbs": achieved_gbs / 8000.0},
+            "e2e": {"value": world * T * e2e_steps / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "dense_ffn": {"us": dense_ms * 1e3, "tokens_per_s": T / (dense_ms * 1e-3),
+                          "what": "torch bf16: silu(x W_in_cat^T) W_out_cat^T, d_ff = E*d_e"},
+            "clocks": clock_info,
+        }
+        if graph_err:
+            line["graph_error"] = graph_err
+        if cb is not None:
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

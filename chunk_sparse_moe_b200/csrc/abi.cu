@@ -1,0 +1,324 @@
+// abi.cu -- the C ABI of libblockffn (include/blockffn.h): argument checks,
+// workspace layout, TMA descriptors and kernel launches.  Nothing here computes
+// on the host; every step of the layer runs in the kernels.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/blockffn.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+using namespace bffn;
+
+std::atomic<unsigned long long> g_wait_ns{2000000000ull};
+std::atomic<int> g_skip_flag{-1};
+thread_local char g_msg[512] = "";
+
+blockffn_status fail(blockffn_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+blockffn_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(BLOCKFFN_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms_current() {
+    static int cache[64];
+    static std::once_flag once[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    std::call_once(once[dev], [dev]() {
+        int v = 0;
+        cache[dev] = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? v : -1;
+    });
+    return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous), box {64, box_outer}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {64, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Layout {
+    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, cntB, flags, partA, partB, hbuf;
+    size_t total;
+    int C, N, MT, RT, KB, KBe;
+    long long Pmax;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_router, int G,
+                 Layout& L) {
+    L.C = (T + n - 1) / n;
+    L.N = bf16 ? (n <= 16 ? 16 : 32) : n;
+    L.MT = bf16 ? d_e / 128 : 1;
+    L.RT = bf16 ? d_h / 128 : 1;
+    L.KB = bf16 ? d_h / 64 : 1;
+    L.KBe = bf16 ? d_e / 64 : 1;
+    L.Pmax = (long long)L.C * E;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + (bytes > 0 ? bytes : 1), 256);
+        return o;
+    };
+    const size_t C = (size_t)L.C, Pm = (size_t)L.Pmax;
+    L.ctl = take(sizeof(Ctl));
+    L.counts = take(C * 4);
+    L.offsets = take((C + 1) * 4);
+    L.idx = take(C * E * 4);
+    L.tmask = take(C * E * 4);
+    L.pair_ce = take(Pm * 4);
+    L.gates = with_router ? take((size_t)T * E * 4) : 0;
+    if (bf16) {
+        L.cntA = take(Pm * L.MT * 4);
+        L.cntB = take(C * L.RT * 4);
+        L.flags = take(Pm * L.MT * 4);
+        L.partA = take((size_t)G * 2 * L.N * 128 * 4);
+        L.partB = take((size_t)G * 2 * L.N * 128 * 4);
+        L.hbuf = take(Pm * L.N * d_e * 2);
+    } else {
+        L.cntA = L.cntB = L.flags = L.partA = L.partB = 0;
+        L.hbuf = take(Pm * n * d_e * 4);
+    }
+    L.total = off;
+    return true;
+}
+
+blockffn_status check_shapes(int T, int d_h, int E, int d_e, int n, blockffn_dtype dt) {
+    if (dt != BLOCKFFN_F32 && dt != BLOCKFFN_BF16) return fail(BLOCKFFN_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    if (T < 0) return fail(BLOCKFFN_ERR_INVALID_ARG, "T = %d < 0", T);
+    if (n < 1 || n > 32) return fail(BLOCKFFN_ERR_INVALID_ARG, "chunk length n = %d outside [1, 32]", n);
+    if (E < 1 || E > 256) return fail(BLOCKFFN_ERR_INVALID_ARG, "E = %d outside [1, 256]", E);
+    if (d_h < 1 || d_e < 1) return fail(BLOCKFFN_ERR_INVALID_ARG, "d_h = %d, d_e = %d must be >= 1", d_h, d_e);
+    const long long C = ((long long)T + n - 1) / n;
+    if (C > (1LL << 22)) return fail(BLOCKFFN_ERR_UNSUPPORTED, "too many chunks (%lld)", C);
+    if (dt == BLOCKFFN_BF16) {
+        if (d_h % 128 != 0) return fail(BLOCKFFN_ERR_UNSUPPORTED, "bf16 needs d_h %% 128 == 0 (d_h = %d)", d_h);
+        if (d_e % 128 != 0 || d_e > 512)
+            return fail(BLOCKFFN_ERR_UNSUPPORTED, "bf16 needs d_e in {128, 256, 384, 512} (d_e = %d)", d_e);
+    } else {
+        if (C > 65535) return fail(BLOCKFFN_ERR_UNSUPPORTED, "fp32 path: at most 65535 chunks");
+    }
+    return BLOCKFFN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* blockffn_status_string(blockffn_status s) {
+    switch (s) {
+        case BLOCKFFN_OK: return "ok";
+        case BLOCKFFN_ERR_INVALID_ARG: return "invalid argument";
+        case BLOCKFFN_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case BLOCKFFN_ERR_CUDA: return "CUDA error";
+        case BLOCKFFN_ERR_TIMEOUT: return "device wait timed out";
+        case BLOCKFFN_ERR_WORKSPACE: return "workspace too small or corrupted";
+    }
+    return "unknown status";
+}
+
+const char* blockffn_last_error_message(void) { return g_msg; }
+
+int blockffn_version(void) { return 100; }
+
+void blockffn_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns > 0 ? ns : 1); }
+
+int blockffn_num_sms(void) { return num_sms_current(); }
+
+void blockffn_debug_skip_flag(int unit) { g_skip_flag.store(unit < 0 ? -1 : unit); }
+
+blockffn_status blockffn_route(const void* x, const void* W_r, const float* b_r,
+                               const float* gamma, float eps, int T, int d_h, int E,
+                               blockffn_dtype dt, float* gates, void* stream) {
+    if (dt != BLOCKFFN_F32 && dt != BLOCKFFN_BF16) return fail(BLOCKFFN_ERR_INVALID_ARG, "unknown dtype");
+    if (T < 0 || d_h < 1 || E < 1 || E > 256) return fail(BLOCKFFN_ERR_INVALID_ARG, "bad shape");
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(BLOCKFFN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    if (dt == BLOCKFFN_BF16 && (d_h % 64 != 0 || E % 16 != 0))
+        return fail(BLOCKFFN_ERR_UNSUPPORTED, "bf16 router needs d_h %% 64 == 0 and E %% 16 == 0");
+    if (T == 0) return BLOCKFFN_OK;
+    if (!x || !W_r || !gamma || !gates) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(W_r) || !aligned16(gates) || !aligned16(gamma) || (b_r && !aligned16(b_r)))
+        return fail(BLOCKFFN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    cudaError_t e = launch_route(x, W_r, b_r, gamma, eps, T, d_h, E, dt == BLOCKFFN_BF16, gates,
+                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "route launch");
+}
+
+blockffn_status blockffn_chunk_union(const float* gates, int T, int E, int n, int32_t* counts,
+                                     int32_t* idx, uint32_t* tmask, void* stream) {
+    if (T < 0 || E < 1 || E > 256 || n < 1 || n > 32) return fail(BLOCKFFN_ERR_INVALID_ARG, "bad shape");
+    if (T == 0) return BLOCKFFN_OK;
+    if (!gates || !counts || !idx || !tmask) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
+    cudaError_t e = launch_chunk_union(gates, T, E, n, counts, idx, tmask, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "chunk_union launch");
+}
+
+size_t blockffn_forward_workspace_bytes(int T, int d_h, int E, int d_e, int n, blockffn_dtype dt,
+                                        int with_router) {
+    if (check_shapes(T, d_h, E, d_e, n, dt) != BLOCKFFN_OK) return 0;
+    const int G = num_sms_current();
+    if (G <= 0) return 0;
+    Layout L;
+    make_layout(T, d_h, E, d_e, n, dt == BLOCKFFN_BF16, with_router != 0, G, L);
+    return L.total;
+}
+
+blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void* stream) {
+    if (!workspace || ws_bytes == 0) return fail(BLOCKFFN_ERR_INVALID_ARG, "null workspace");
+    cudaError_t e = cudaMemsetAsync(workspace, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "workspace memset");
+}
+
+blockffn_status blockffn_forward(const void* x, const float* gates, const void* W_r,
+                                 const float* b_r, const float* gamma, float eps,
+                                 const void* W_in, const void* W_out, int T, int d_h, int E,
+                                 int d_e, int n, blockffn_dtype dt, void* y, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+    blockffn_status st = check_shapes(T, d_h, E, d_e, n, dt);
+    if (st != BLOCKFFN_OK) return st;
+    const bool routed = gates == nullptr;
+    if (routed) {
+        if (!W_r || !gamma) return fail(BLOCKFFN_ERR_INVALID_ARG, "no gates: W_r and gamma are required");
+        if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(BLOCKFFN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+        if (dt == BLOCKFFN_BF16 && E % 16 != 0)
+            return fail(BLOCKFFN_ERR_UNSUPPORTED, "bf16 router needs E %% 16 == 0");
+    } else if (W_r || b_r || gamma) {
+        return fail(BLOCKFFN_ERR_INVALID_ARG, "pass either gates or router weights, not both");
+    }
+    if (T == 0) return BLOCKFFN_OK;
+    if (!x || !W_in || !W_out || !y || !workspace) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(W_in) || !aligned16(W_out) || !aligned16(y) ||
+        !aligned16(workspace) || (gates && !aligned16(gates)) || (W_r && !aligned16(W_r)) ||
+        (gamma && !aligned16(gamma)) || (b_r && !aligned16(b_r)))
+        return fail(BLOCKFFN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    const int G = num_sms_current();
+    if (G <= 0) return fail(BLOCKFFN_ERR_CUDA, "no current CUDA device");
+    const bool bf16 = dt == BLOCKFFN_BF16;
+    Layout L;
+    make_layout(T, d_h, E, d_e, n, bf16, routed, G, L);
+    if (ws_bytes < L.total)
+        return fail(BLOCKFFN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, L.total);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    cudaError_t e;
+
+    const float* g = gates;
+    if (routed) {
+        float* gw = reinterpret_cast<float*>(ws + L.gates);
+        e = launch_route(x, W_r, b_r, gamma, eps, T, d_h, E, bf16, gw, s);
+        if (e != cudaSuccess) return cuda_fail(e, "route launch");
+        g = gw;
+    }
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+    int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+    uint32_t* tmask = reinterpret_cast<uint32_t*>(ws + L.tmask);
+    int32_t* pair_ce = reinterpret_cast<int32_t*>(ws + L.pair_ce);
+
+    if (!bf16) {
+        e = launch_chunk_union_plan(g, T, E, n, counts, idx, tmask, offsets, pair_ce, y, d_h, 4, s);
+        if (e != cudaSuccess) return cuda_fail(e, "union launch");
+        e = launch_forward_f32(static_cast<const float*>(x), g, static_cast<const float*>(W_in),
+                               static_cast<const float*>(W_out), counts, offsets, pair_ce, tmask,
+                               reinterpret_cast<float*>(ws + L.hbuf), T, d_h, E, d_e, n,
+                               static_cast<float*>(y), G, s);
+        return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "fp32 forward launch");
+    }
+
+    const bool fuse = L.C == 1;
+    if (!fuse) {
+        e = launch_chunk_union_plan(g, T, E, n, counts, idx, tmask, offsets, pair_ce, y, d_h, 2, s);
+        if (e != cudaSuccess) return cuda_fail(e, "union launch");
+    }
+    CUtensorMap maps[4];
+    if (!make_map(&maps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
+        !make_map(&maps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
+        !make_map(&maps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
+        !make_map(&maps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)L.Pmax * L.N, (uint32_t)L.N))
+        return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    TcArgs a;
+    a.gates = g;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.pair_ce = pair_ce;
+    a.tmask = tmask;
+    a.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
+    a.partA = reinterpret_cast<float*>(ws + L.partA);
+    a.partB = reinterpret_cast<float*>(ws + L.partB);
+    a.cntA = reinterpret_cast<uint32_t*>(ws + L.cntA);
+    a.cntB = reinterpret_cast<uint32_t*>(ws + L.cntB);
+    a.flags = reinterpret_cast<uint32_t*>(ws + L.flags);
+    a.ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
+    a.y = static_cast<__nv_bfloat16*>(y);
+    a.T = T;
+    a.d_h = d_h;
+    a.E = E;
+    a.d_e = d_e;
+    a.n = n;
+    a.N = L.N;
+    a.C = L.C;
+    a.KB = L.KB;
+    a.MT = L.MT;
+    a.RT = L.RT;
+    a.KBe = L.KBe;
+    a.fuse_union = fuse ? 1 : 0;
+    a.wait_ns = g_wait_ns.load();
+    a.skip_flag_unit = g_skip_flag.load();
+    e = launch_forward_tc(a, maps, G, s);
+    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "tensor-core forward launch");
+}
+
+blockffn_status blockffn_get_device_status(const void* workspace, void* stream, int32_t* detail) {
+    if (!workspace) return fail(BLOCKFFN_ERR_INVALID_ARG, "null workspace");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t h[2] = {0, 0};
+    cudaError_t e = cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "device status read");
+    if (detail) *detail = h[1];
+    return static_cast<blockffn_status>(h[0]);
+}
+
+}  // extern "C"

@@ -1,0 +1,105 @@
+// common.cuh -- shared definitions of the BlockFFN CUDA library: workspace
+// control block, device-side error recording and bounded waits.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace bffn {
+
+// Status codes, identical to blockffn_status in include/blockffn.h.
+enum : int32_t {
+    kOk = 0,
+    kErrInvalidArg = 1,
+    kErrUnsupported = 2,
+    kErrCuda = 3,
+    kErrTimeout = 4,
+    kErrWorkspace = 5,
+};
+
+// Which wait ran out (the "detail" of a timeout).
+enum : int32_t {
+    kWaitEmpty = 1,      // producer waiting for a free pipeline stage
+    kWaitFullW = 2,      // MMA waiting for a weight/activation tile
+    kWaitFullH = 3,      // MMA waiting for a gated-activation tile
+    kWaitAccFull = 4,    // epilogue waiting for an accumulator
+    kWaitAccEmpty = 5,   // MMA waiting for a free accumulator
+    kWaitFlag = 6,       // activation loader waiting for another block's result
+    kWaitDrain = 7,      // teardown waiting for its own copies in flight
+    kWaitMmaDone = 8,    // teardown waiting for the last MMAs
+};
+
+// Control block at offset 0 of every forward workspace (256 bytes reserved).
+struct Ctl {
+    int32_t status;        // first device-side error (sticky until reset)
+    int32_t detail;        // which wait / check
+    uint32_t epoch;        // number of completed forward launches (flag stamp)
+    uint32_t done;         // thread blocks of the current launch that finished
+    uint32_t pad[60];
+};
+static_assert(sizeof(Ctl) == 256, "control block is 256 bytes");
+
+__device__ __forceinline__ void record_error(Ctl* ctl, int32_t code, int32_t detail) {
+    if (atomicCAS(&ctl->status, 0, code) == 0) atomicExch(&ctl->detail, detail);
+}
+
+// Spin on an mbarrier phase for at most limit_ns.  Gives up early when another
+// role of the block has aborted.  On running out, records a timeout and sets
+// the block's abort flag.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                         volatile int* abort, Ctl* ctl, int32_t detail) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_error(ctl, kErrTimeout, detail);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// Same, without the abort short-cut: used at teardown to let copies land.
+__device__ __forceinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity,
+                                               uint64_t limit_ns, Ctl* ctl) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_error(ctl, kErrTimeout, kWaitDrain);
+            return false;
+        }
+    }
+}
+
+// Spin until *flag == want (acquire), bounded.
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t want, uint64_t limit_ns,
+                                          volatile int* abort, Ctl* ctl) {
+    if (ld_acquire_gpu(flag) == want) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(flag) == want) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_error(ctl, kErrTimeout, kWaitFlag);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__host__ __device__ inline long long ceil_div_ll(long long a, long long b) {
+    return (a + b - 1) / b;
+}
+
+}  // namespace bffn

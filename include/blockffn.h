@@ -1,0 +1,188 @@
+/*
+ * blockffn.h -- C ABI of the BlockFFN chunk-union layer forward on B200 (sm_100a).
+ *
+ * The layer (pages: "BlockFFN: Sparse Mixture-of-Experts Optimized for End-Device
+ * Deployment", sections Core Concept and Architecture Overview; "BlockFFN: Towards
+ * End-Side Acceleration-Friendly Mixture-of-Experts with Chunk-Level Activation
+ * Sparsity", Abstract):
+ *
+ *   route:  g[t,:] = RMSNorm(ReLU(W_r x_t + b_r))          over the E experts
+ *   union:  U_c    = { e : g[t,e] != 0 for some t in chunk c }, chunks of n tokens
+ *   expert: o_e(x) = W_out_e Swish(W_in_e x)                non-gated, d_e << d_h
+ *   output: y[t,:] = sum_{e in U_c, ascending} [g[t,e] != 0] g[t,e] o_e(x_t)
+ *
+ * Only the union experts run, each over every token of the chunk as one small
+ * dense GEMM pair; tokens whose own gate is zero are masked after computing.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *   row-major, 16-byte aligned.  The library allocates no device memory; scratch
+ *   space comes from the caller's workspace (blockffn_forward_workspace_bytes).
+ * - Weights follow the nn.Linear convention weight[out, in]:
+ *     x [T, d_h]; W_r [E, d_h]; b_r [E] fp32; gamma [E] fp32; gates [T, E] fp32;
+ *     W_in [E, d_e, d_h]; W_out [E, d_h, d_e]; y [T, d_h].
+ *   x, W_r, W_in, W_out and y share one element type (blockffn_dtype).
+ * - Chunks are n consecutive tokens starting at token 0; C = ceil(T / n); the
+ *   last chunk may be short (its missing tokens count as inactive).  n in [1, 32].
+ * - stream is a cudaStream_t (NULL = the legacy default stream).  Every call is
+ *   asynchronous on it, except blockffn_get_device_status, which synchronizes it.
+ * - Arguments are validated on the host before anything is launched; a call that
+ *   returns an error other than BLOCKFFN_ERR_CUDA has launched nothing.
+ * - Device-side failures (a bounded wait that ran out, a corrupted workspace) are
+ *   recorded in the workspace status word and read by blockffn_get_device_status.
+ *   After one, reset the workspace before the next call.
+ * - Results are deterministic: two calls with the same inputs, shapes and device
+ *   give bit-identical outputs (every sum runs in a fixed order).
+ */
+#ifndef BLOCKFFN_H
+#define BLOCKFFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BLOCKFFN_OK = 0,
+    BLOCKFFN_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer      */
+    BLOCKFFN_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement   */
+    BLOCKFFN_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed     */
+    BLOCKFFN_ERR_TIMEOUT = 4,     /* device: a bounded wait ran out (status word)    */
+    BLOCKFFN_ERR_WORKSPACE = 5    /* workspace too small, or found corrupted         */
+} blockffn_status;
+
+typedef enum {
+    BLOCKFFN_F32 = 0,  /* fp32 values, fp32 arithmetic (CUDA-core FFMA)               */
+    BLOCKFFN_BF16 = 1  /* bf16 values, fp32 accumulation (tcgen05 tensor cores)       */
+} blockffn_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* blockffn_status_string(blockffn_status s);
+
+/* Text of the last host-side error of the calling thread ("" when none):
+ * which check failed, or the CUDA error string.  Valid until the next call. */
+const char* blockffn_last_error_message(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int blockffn_version(void);
+
+/*
+ * blockffn_route -- the router.
+ * Pages: "BlockFFN: Sparse Mixture-of-Experts Optimized for End-Device Deployment",
+ * Architecture Overview (Router Module: linear map, ReLU, RMSNorm) and Router
+ * Architecture Setup (nn.Linear without bias, nn.RMSNorm over the experts).
+ *
+ *   logit[t,e] = sum_k W_r[e,k] x[t,k] + (b_r ? b_r[e] : 0)      (fp32 accumulation)
+ *   r          = max(logit, 0)
+ *   gates[t,e] = r > 0 ? gamma[e] * r / sqrt(mean_e' r[t,e']^2 + eps) : 0
+ *
+ * x [T, d_h] and W_r [E, d_h] in dtype dt; b_r [E] fp32 or NULL; gamma [E] fp32;
+ * eps >= 0.  gates [T, E] fp32 output.  Requirements: T >= 0, 1 <= E <= 256,
+ * d_h >= 1; bf16 additionally d_h % 64 == 0 and E % 16 == 0.
+ */
+blockffn_status blockffn_route(const void* x, const void* W_r, const float* b_r,
+                               const float* gamma, float eps, int T, int d_h, int E,
+                               blockffn_dtype dt, float* gates, void* stream);
+
+/*
+ * blockffn_chunk_union -- the union of active experts of each n-token chunk.
+ * Pages: "BlockFFN: Sparse Mixture-of-Experts Optimized for End-Device Deployment",
+ * Core Concept and Architecture Overview (the kernel computes only the union of
+ * the experts activated across n tokens).
+ *
+ *   tmask[c,e]  bit j set  <=>  t = c*n + j < T and gates[t,e] != 0  (IEEE !=)
+ *   counts[c]   = number of e with tmask[c,e] != 0
+ *   idx[c,s]    = the s-th such e in ascending order for s < counts[c], else -1
+ *
+ * gates [T, E] fp32 (finite); outputs counts [C] int32, idx [C, E] int32,
+ * tmask [C, E] uint32.  Requirements: T >= 0, 1 <= E <= 256, 1 <= n <= 32.
+ * Integer results, bit-exact.
+ */
+blockffn_status blockffn_chunk_union(const float* gates, int T, int E, int n,
+                                     int32_t* counts, int32_t* idx, uint32_t* tmask,
+                                     void* stream);
+
+/*
+ * blockffn_forward_workspace_bytes -- size of the scratch buffer blockffn_forward
+ * needs for these shapes (0 when the shapes are invalid).  with_router != 0 when
+ * the gates will come from the router (the workspace then also holds them).
+ */
+size_t blockffn_forward_workspace_bytes(int T, int d_h, int E, int d_e, int n,
+                                        blockffn_dtype dt, int with_router);
+
+/*
+ * blockffn_workspace_reset -- zero a workspace (asynchronous memset on stream).
+ * Required once before a workspace's first use and after any device-side error.
+ */
+blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * blockffn_forward -- the layer output y over all chunks.
+ * Pages: "BlockFFN: Sparse Mixture-of-Experts Optimized for End-Device Deployment",
+ * Core Concept (union of activated experts over n tokens, unneeded activations
+ * masked after computation), Architecture Overview (non-gated Swish experts),
+ * Full BlockFFN Layer with Combined Losses (gate times expert output, summed over
+ * experts).
+ *
+ * Gating source, exactly one of:
+ *   gates != NULL : injected gates [T, E] fp32 (W_r, b_r, gamma ignored, must be NULL);
+ *   gates == NULL : the router runs first (W_r, gamma required, b_r optional, eps).
+ * W_in [E, d_e, d_h] and W_out [E, d_h, d_e] in dtype dt; y [T, d_h] in dtype dt is
+ * fully overwritten (rows of tokens with no active expert are exact zeros).
+ * workspace: ws_bytes >= blockffn_forward_workspace_bytes(...), reset once with
+ * blockffn_workspace_reset; it carries state between calls (never share one
+ * workspace between calls that may overlap on the GPU).
+ * Requirements: T >= 0, 1 <= n <= 32, 1 <= E <= 256;
+ *   bf16: d_h % 128 == 0, d_e % 128 == 0, d_e <= 512, E % 16 == 0 when routed;
+ *   fp32: any d_h, d_e >= 1.
+ * Arithmetic: bf16 inputs, fp32 accumulation; the gated Swish activations are
+ * rounded to bf16 between the two GEMMs; y is rounded once to dt.
+ */
+blockffn_status blockffn_forward(const void* x, const float* gates, const void* W_r,
+                                 const float* b_r, const float* gamma, float eps,
+                                 const void* W_in, const void* W_out, int T, int d_h,
+                                 int E, int d_e, int n, blockffn_dtype dt, void* y,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * blockffn_get_device_status -- synchronize stream, then read the device status
+ * word of a workspace: BLOCKFFN_OK, or the first device-side error recorded
+ * (BLOCKFFN_ERR_TIMEOUT, BLOCKFFN_ERR_WORKSPACE).  detail (may be NULL) receives
+ * a code naming the wait that ran out.  Returns BLOCKFFN_ERR_CUDA if the
+ * synchronization itself failed.
+ */
+blockffn_status blockffn_get_device_status(const void* workspace, void* stream,
+                                           int32_t* detail);
+
+/*
+ * blockffn_set_wait_limit_ns -- upper bound, in nanoseconds, of every spin-wait
+ * inside the kernels (waits on another thread block's result or on a copy).  A
+ * wait that runs out records BLOCKFFN_ERR_TIMEOUT and the kernel returns.  The
+ * default is 2e9 (2 s), far above any legitimate wait.  Applies to later launches.
+ */
+void blockffn_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * blockffn_debug_skip_flag -- failure-detection test support.  For later forward
+ * launches (bf16 path), the thread block that finishes expert-in unit `unit`
+ * (the unit index is pair * (d_e / 128) + m-tile) writes its activations but
+ * never publishes the flag that says so; the expert-out tiles that need them
+ * then wait until the bounded-wait limit runs out, and the launch records
+ * BLOCKFFN_ERR_TIMEOUT in the workspace.  -1 (the default) turns it off.
+ */
+void blockffn_debug_skip_flag(int unit);
+
+/*
+ * blockffn_num_sms -- streaming multiprocessors of the current device (the grid
+ * size of the persistent forward kernel), or -1 on error.
+ */
+int blockffn_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BLOCKFFN_H */

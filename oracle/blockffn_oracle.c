@@ -198,23 +198,20 @@ void oracle_forward_chunk_union(const double* x, const double* gates, const doub
     uint32_t* tmask = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)C * E);
     oracle_chunk_union(gates, T, E, n, counts, idx, tmask);
     memset(y, 0, sizeof(double) * (size_t)T * d_h);
-    int c;
+    int t;
 #pragma omp parallel for schedule(dynamic, 1)
-    for (c = 0; c < C; ++c) {
+    for (t = 0; t < T; ++t) {
+        int c = t / n, j = t % n;
         double* h = (double*)malloc(sizeof(double) * (size_t)d_e);
         double* o = (double*)malloc(sizeof(double) * (size_t)d_h);
         for (int s = 0; s < counts[c]; ++s) {
             int e = idx[(size_t)c * E + s];
             uint32_t bits = tmask[(size_t)c * E + e];
-            for (int j = 0; j < n; ++j) {
-                int t = c * n + j;
-                if (t >= T) break;
-                expert_apply(x + (size_t)t * d_h, W_in, W_out, d_h, d_e, e, h, o);
-                int keep = (int)((bits >> j) & 1u);
-                double g = gates[(size_t)t * E + e];
-                for (int i = 0; i < d_h; ++i)
-                    y[(size_t)t * d_h + i] += keep ? g * o[i] : 0.0;
-            }
+            expert_apply(x + (size_t)t * d_h, W_in, W_out, d_h, d_e, e, h, o);
+            int keep = (int)((bits >> j) & 1u);
+            double g = gates[(size_t)t * E + e];
+            for (int i = 0; i < d_h; ++i)
+                y[(size_t)t * d_h + i] += keep ? g * o[i] : 0.0;
         }
         free(h);
         free(o);

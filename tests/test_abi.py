@@ -1,0 +1,98 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+include/blockffn.h declares, and rejects bad arguments on the host before any
+CUDA call (no compute runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "blockffn.h")
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(blockffn_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from chunk_sparse_moe_b200 import build
+    build.build()
+    from chunk_sparse_moe_b200 import _lib
+    return _lib
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for must in ("blockffn_route", "blockffn_chunk_union", "blockffn_forward",
+                 "blockffn_forward_workspace_bytes", "blockffn_get_device_status"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), f"{name} declared in blockffn.h but not exported"
+        assert name in lib.SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.lib.blockffn_status_string(code)
+    assert lib.lib.blockffn_version() >= 100
+
+
+@pytest.mark.parametrize("T,d_h,E,d_e,n,dt", [
+    (32, 2048, 64, 128, 0, 1),      # n < 1
+    (32, 2048, 64, 128, 33, 1),     # n > 32
+    (32, 2048, 0, 128, 32, 1),      # E < 1
+    (32, 2048, 257, 128, 32, 1),    # E > 256
+    (-1, 2048, 64, 128, 32, 1),     # T < 0
+    (32, 2000, 64, 128, 32, 1),     # bf16 d_h % 128
+    (32, 2048, 64, 64, 32, 1),      # bf16 d_e % 128
+    (32, 2048, 64, 1024, 32, 1),    # bf16 d_e > 512
+    (32, 2048, 64, 128, 32, 7),     # unknown dtype
+])
+def test_forward_rejects_bad_shapes_on_host(lib, T, d_h, E, d_e, n, dt):
+    L = lib.lib
+    assert L.blockffn_forward_workspace_bytes(T, d_h, E, d_e, n, dt, 0) == 0
+    st = L.blockffn_forward(16, 16, None, None, None, 0.0, 16, 16, T, d_h, E, d_e, n, dt, 16, 16,
+                            1 << 30, None)
+    assert st in (lib.ERR_INVALID_ARG, lib.ERR_UNSUPPORTED)
+    assert L.blockffn_last_error_message()
+
+
+def test_forward_gating_source_is_exclusive(lib):
+    L = lib.lib
+    # gates and router weights together
+    st = L.blockffn_forward(16, 16, 16, None, None, 0.0, 16, 16, 32, 2048, 64, 128, 32, 1, 16, 16,
+                            1 << 30, None)
+    assert st == lib.ERR_INVALID_ARG
+    # neither
+    st = L.blockffn_forward(16, None, None, None, None, 0.0, 16, 16, 32, 2048, 64, 128, 32, 1, 16,
+                            16, 1 << 30, None)
+    assert st == lib.ERR_INVALID_ARG
+
+
+def test_union_and_route_reject_bad_args(lib):
+    L = lib.lib
+    assert L.blockffn_chunk_union(16, 32, 64, 0, 16, 16, 16, None) == lib.ERR_INVALID_ARG
+    assert L.blockffn_chunk_union(16, 32, 300, 8, 16, 16, 16, None) == lib.ERR_INVALID_ARG
+    assert L.blockffn_chunk_union(None, 32, 64, 8, 16, 16, 16, None) == lib.ERR_INVALID_ARG
+    assert L.blockffn_route(16, 16, None, 16, -1.0, 32, 64, 16, 1, 16, None) == lib.ERR_INVALID_ARG
+    assert L.blockffn_route(16, 16, None, 16, 0.0, 32, 60, 16, 1, 16, None) == lib.ERR_UNSUPPORTED
+    # misaligned pointers
+    assert L.blockffn_route(17, 16, None, 16, 0.0, 32, 64, 16, 1, 16, None) == lib.ERR_INVALID_ARG
+
+
+def test_empty_inputs_are_no_ops(lib):
+    L = lib.lib
+    # T = 0: nothing to do, nothing launched, no pointer needed
+    assert L.blockffn_chunk_union(None, 0, 64, 32, None, None, None, None) == lib.OK
+    assert L.blockffn_route(None, None, None, None, 0.0, 0, 64, 16, 1, None, None) == lib.OK
+    assert L.blockffn_forward(None, 16, None, None, None, 0.0, None, None, 0, 2048, 64, 128, 32,
+                              1, None, None, 0, None) == lib.OK

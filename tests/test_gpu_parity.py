@@ -1,0 +1,209 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.
+
+* chunk union: bit-exact counts / index lists / token masks;
+* router: gate-zero masks bit-exact outside the fp32 rounding band of the logit,
+  gate values to fp32 accuracy;
+* forward: bf16 max |dy| <= 1e-2 max|y_ref| and relative L2 <= 5e-3, fp32
+  relative L2 <= 1e-5; rows of tokens with no active expert exactly zero;
+* the five workloads at full size (whole outputs where the oracle is quick,
+  whole sampled chunks where it is not), small shapes that span several tiles
+  with ragged tails, and the degenerate cases (empty union, one expert, all
+  experts, T = 0, one token);
+* determinism and workspace reuse.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from gpu_common import (assert_close, chunk_tokens, dev, oracle_y, require_cuda,
+                        router_mask_band, run_gpu, to_np64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bffn():
+    return require_cuda()
+
+
+# ------------------------------------------------------------ chunk union --
+
+def _union_case(seed, T, E, n, p_on=0.3):
+    rng = np.random.default_rng(seed)
+    g = np.where(rng.random((T, E)) < p_on, rng.standard_normal((T, E)), 0.0).astype(np.float32)
+    g[rng.random((T, E)) < 0.05] = -0.0      # negative zero counts as inactive
+    return g
+
+
+@pytest.mark.parametrize("T,E,n", [(32, 64, 32), (70, 16, 32), (1, 1, 1), (33, 256, 32),
+                                   (100, 128, 8), (7, 3, 7), (4096, 64, 32), (257, 40, 31),
+                                   (64, 64, 1)])
+def test_chunk_union_bit_exact(bffn, T, E, n):
+    g = _union_case(T * 1000 + E + n, T, E, n)
+    counts, idx, tmask = bffn.chunk_union(dev(g, torch.float32), n)
+    rc, ri, rt = oracle.chunk_union(g, n)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+    assert np.array_equal(tmask.cpu().numpy().view(np.uint32), rt)
+
+
+def test_chunk_union_markov_workload(bffn):
+    w = wl.chunk32()
+    counts, idx, tmask = bffn.chunk_union(dev(w.gates, torch.float32), w.n)
+    rc, ri, rt = oracle.chunk_union(w.gates, w.n)
+    assert np.array_equal(counts.cpu().numpy(), rc) and np.array_equal(idx.cpu().numpy(), ri)
+    assert np.array_equal(tmask.cpu().numpy().view(np.uint32), rt)
+
+
+# ----------------------------------------------------------------- router --
+
+def _check_route(bffn, w):
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    x, W_r = dev(w.x, dt), dev(w.W_r, dt)
+    b = None if w.b_r is None else dev(w.b_r, torch.float32)
+    g = to_np64(bffn.route(x, W_r, dev(w.gamma, torch.float32), w.eps, b_r=b))
+    logits, g_ref = oracle.route(w.x, w.W_r, w.gamma, w.eps, b_r=w.b_r)
+    band = router_mask_band(w)
+    sure = np.abs(logits) > band
+    assert np.array_equal((g != 0)[sure], (g_ref != 0)[sure]), "gate-zero mask differs"
+    assert np.sum(~sure) <= max(1, int(1e-3 * g.size)), "too many logits inside the band"
+    # values: fp32 accumulation and normalisation
+    both = (g != 0) & (g_ref != 0)
+    err = np.max(np.abs(g - g_ref)[both]) if np.any(both) else 0.0
+    assert err <= 1e-4 * max(1.0, float(np.max(np.abs(g_ref)))), f"gate values off by {err}"
+    return g
+
+
+def test_route_tiny_f32(bffn):
+    _check_route(bffn, wl.tiny_f32())
+
+
+def test_route_seq4096_bf16(bffn):
+    _check_route(bffn, wl.seq4096())
+
+
+def test_route_edge_rows(bffn):
+    """A row whose logits are all <= 0 gives zero gates; negative gamma keeps the sign."""
+    w = wl.make_routed("edge", 40, 8, 128, 16, 128, "bf16", seed=3, bias_shift=-0.8)
+    w.x[0] = 0.0                     # logits = bias < 0 -> all gates 0
+    w.gamma = np.linspace(-1.0, 1.5, 16).astype(np.float32)
+    g = _check_route(bffn, w)
+    assert not np.any(g[0])
+
+
+# ---------------------------------------------------------------- forward --
+
+def test_forward_tiny_f32_router(bffn):
+    w = wl.tiny_f32()
+    y, g = run_gpu(w)
+    assert_close(y, oracle.forward_dense(w.x, g, w.W_in, w.W_out), "f32", "tiny_f32")
+
+
+@pytest.mark.parametrize("T,n,d_h,E,d_e,regime", [
+    (32, 32, 128, 1, 128, "all_on"),       # one expert, one tile each way
+    (32, 32, 256, 4, 128, "markov80"),
+    (70, 32, 512, 16, 128, "markov80"),    # 3 chunks, ragged 6-token tail
+    (70, 32, 512, 16, 256, "bern0.2"),     # two 128-row tiles per expert
+    (45, 8, 384, 16, 128, "markov80"),     # N = 16 tokens per MMA, ragged
+    (5, 1, 256, 8, 128, "bern0.2"),        # one-token chunks
+    (1, 32, 256, 8, 128, "all_on"),        # one token in a 32-token chunk
+    (96, 32, 1024, 64, 128, "markov90"),
+    (40, 17, 256, 32, 384, "markov80"),    # d_e = 384, n = 17 (N = 32)
+])
+def test_forward_bf16_small(bffn, T, n, d_h, E, d_e, regime):
+    w = wl.make_injected("small", T, n, d_h, E, d_e, "bf16", regime, seed=T + d_h + E)
+    y, g = run_gpu(w)
+    assert_close(y, oracle_y(w, g), "bf16", f"T{T} n{n} d_h{d_h} E{E} d_e{d_e} {regime}")
+
+
+def test_forward_bf16_dense_matches_dense_definition(bffn):
+    """All gates on: the union is every expert; compare with the dense definition."""
+    w = wl.make_injected("dense", 32, 32, 256, 8, 128, "bf16", "all_on", seed=4)
+    y, g = run_gpu(w)
+    assert_close(y, oracle.forward_dense(w.x, g, w.W_in, w.W_out), "bf16", "all_on dense")
+
+
+def test_forward_empty_union_is_zero(bffn):
+    for T, n in ((32, 32), (70, 32)):
+        w = wl.make_injected("off", T, n, 256, 16, 128, "bf16", "all_off", seed=1)
+        y, _ = run_gpu(w)
+        assert not np.any(y)
+
+
+def test_forward_partly_empty_chunks(bffn):
+    w = wl.make_injected("mixed", 96, 32, 256, 16, 128, "bf16", "markov80", seed=2)
+    w.gates[32:64] = 0.0            # middle chunk has an empty union
+    y, g = run_gpu(w)
+    assert not np.any(y[32:64])
+    assert_close(y, oracle_y(w, g), "bf16", "mixed")
+
+
+def test_forward_router_bf16_small(bffn):
+    w = wl.make_routed("r", 100, 32, 256, 16, 128, "bf16", seed=5, bias_shift=-0.8, ar_rho=0.95)
+    y, g = run_gpu(w)
+    assert_close(y, oracle_y(w, g), "bf16", "router small")
+
+
+def test_forward_zero_tokens(bffn):
+    W_in = torch.zeros((4, 128, 256), dtype=torch.bfloat16, device="cuda")
+    W_out = torch.zeros((4, 256, 128), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((0, 256), dtype=torch.bfloat16, device="cuda")
+    g = torch.zeros((0, 4), dtype=torch.float32, device="cuda")
+    y = bffn.forward(x, W_in, W_out, 32, gates=g, workspace=bffn.Workspace(256))
+    assert y.shape == (0, 256)
+
+
+def test_deterministic_and_workspace_reuse(bffn):
+    w = wl.chunk32()
+    ws = bffn.Workspace.for_shapes(w.T, w.d_h, w.E, w.d_e, w.n, torch.bfloat16, False)
+    y1, g = run_gpu(w, ws)
+    y2, _ = run_gpu(w, ws)
+    assert np.array_equal(y1, y2), "two calls differ"
+    w2 = wl.chunk32(weights=(w.W_in, w.W_out), x_seed=77)
+    y3, g3 = run_gpu(w2, ws)
+    assert_close(y3, oracle_y(w2, g3), "bf16", "reuse")
+    y4, _ = run_gpu(w, ws)
+    assert np.array_equal(y1, y4)
+    assert bffn.device_status(ws) == (0, 0)
+
+
+# ----------------------------------------------- the five workloads, full size --
+
+def test_workload_tiny_f32(bffn):
+    w = wl.tiny_f32()
+    y, g = run_gpu(w)
+    assert_close(y, oracle.forward_dense(w.x, g, w.W_in, w.W_out), "f32", "tiny_f32")
+
+
+def test_workload_chunk32_full(bffn):
+    w = wl.chunk32()
+    y, g = run_gpu(w)
+    assert_close(y, oracle.forward_dense(w.x, g, w.W_in, w.W_out), "bf16", "chunk32")
+
+
+def test_workload_batch16_sampled_chunks(bffn):
+    w = wl.batch16()
+    y, g = run_gpu(w)
+    tok = chunk_tokens(w, [0, 7, 15])
+    assert_close(y[tok], oracle_y(w, g, tok), "bf16", "batch16")
+
+
+def test_workload_seq4096_sampled_chunks(bffn):
+    w = wl.seq4096()
+    y, g = run_gpu(w)
+    tok = chunk_tokens(w, [0, 64, 127])
+    assert_close(y[tok], oracle_y(w, g, tok), "bf16", "seq4096")
+    # every row: zero exactly where no expert is active
+    assert np.array_equal(np.any(y != 0, axis=1), np.any(g != 0, axis=1))
+
+
+@pytest.mark.parametrize("n", wl.SWEEP_CHUNKS)
+@pytest.mark.parametrize("regime", wl.SWEEP_REGIMES)
+def test_workload_sweep_first_chunk(bffn, n, regime):
+    """d_h=4096, E=128: one decode-step call on the sequence's first chunk."""
+    w = wl.sweep(n, regime, T=n)
+    y, g = run_gpu(w)
+    assert_close(y, oracle_y(w, g), "bf16", f"sweep n{n} {regime}")

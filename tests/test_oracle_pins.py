@@ -311,8 +311,8 @@ MUTANTS = {
     # the union schedule reads the chunk's first token's gate for every token
     # (skipping the post-hoc mask alone is an equivalent mutant for finite
     # inputs: a zero gate already zeroes the term)
-    "wrong_token_gate": ("int keep = (int)((bits >> j) & 1u);\n                double g = gates[(size_t)t * E + e];",
-                         "int keep = (int)((bits >> j) & 1u);\n                double g = gates[(size_t)(c * n) * E + e];"),
+    "wrong_token_gate": ("int keep = (int)((bits >> j) & 1u);\n            double g = gates[(size_t)t * E + e];",
+                         "int keep = (int)((bits >> j) & 1u);\n            double g = gates[(size_t)(c * n) * E + e];"),
     # RMS over the wrong count (sum instead of mean)
     "rms_sum": ("ms /= (double)E;", "ms /= 1.0;"),
     # union bitmask off by one token
