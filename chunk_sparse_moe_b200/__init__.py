@@ -5,8 +5,10 @@ CUDA torch tensors, check them, and pass raw device pointers and the current
 CUDA stream to the C ABI (include/blockffn.h).  All arithmetic runs in the
 library's kernels; PyTorch only provides device memory and streams.
 """
-from .api import (BlockFFNError, Workspace, chunk_union, debug_skip_flag, device_status, forward,
+from .api import (BlockFFNError, Workspace, chunk_union, debug_set_trace, debug_skip_flag, device_status,
+                  forward,
                   num_sms, route, set_wait_limit_ns, version, workspace_bytes)
 
-__all__ = ["BlockFFNError", "Workspace", "chunk_union", "debug_skip_flag", "device_status",
+__all__ = ["BlockFFNError", "Workspace", "chunk_union", "debug_set_trace", "debug_skip_flag",
+           "device_status",
            "forward", "num_sms", "route", "set_wait_limit_ns", "version", "workspace_bytes"]

@@ -42,6 +42,7 @@ SIGNATURES = {
     "blockffn_set_wait_limit_ns": (None, [c_uint64]),
     "blockffn_num_sms": (c_int, []),
     "blockffn_debug_skip_flag": (None, [c_int]),
+    "blockffn_debug_set_trace": (None, [c_void_p]),
 }
 
 for _name, (_res, _args) in SIGNATURES.items():

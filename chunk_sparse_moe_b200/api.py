@@ -65,6 +65,14 @@ def debug_skip_flag(unit: int) -> None:
     lib.blockffn_debug_skip_flag(int(unit))
 
 
+def debug_set_trace(buf: Optional[torch.Tensor]) -> None:
+    """Attach (or detach with None) a zeroed int64 CUDA tensor of num_sms()*32
+    entries that later bf16 forward launches fill with per-block timestamps."""
+    if buf is not None and (buf.dtype != torch.int64 or buf.numel() < 32 * num_sms()):
+        raise ValueError("trace buffer: int64 tensor of at least num_sms()*32 entries")
+    lib.blockffn_debug_set_trace(None if buf is None else _ptr(buf))
+
+
 def route(x: torch.Tensor, W_r: torch.Tensor, gamma: torch.Tensor, eps: float,
           b_r: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """gates [T, E] fp32 = RMSNorm(ReLU(x W_r^T + b_r)) over the experts."""

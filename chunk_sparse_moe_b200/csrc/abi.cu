@@ -23,6 +23,7 @@ using namespace bffn;
 
 std::atomic<unsigned long long> g_wait_ns{2000000000ull};
 std::atomic<int> g_skip_flag{-1};
+std::atomic<unsigned long long*> g_trace{nullptr};
 thread_local char g_msg[512] = "";
 
 blockffn_status fail(blockffn_status st, const char* fmt, ...) {
@@ -79,7 +80,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 }
 
 struct Layout {
-    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, cntB, flags, partA, partB, hbuf;
+    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, readyA, cntB, partA, partB, hbuf;
     size_t total;
     int C, N, MT, RT, KB, KBe;
     long long Pmax;
@@ -111,14 +112,14 @@ bool make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
     L.pair_ce = take(Pm * 4);
     L.gates = with_router ? take((size_t)T * E * 4) : 0;
     if (bf16) {
-        L.cntA = take(Pm * L.MT * 4);
-        L.cntB = take(C * L.RT * 4);
-        L.flags = take(Pm * L.MT * 4);
+        L.cntA = take(2 * Pm * L.MT * 4);
+        L.readyA = take(2 * Pm * L.MT * 4);
+        L.cntB = take(2 * C * L.RT * 4);
         L.partA = take((size_t)G * 2 * L.N * 128 * 4);
         L.partB = take((size_t)G * 2 * L.N * 128 * 4);
         L.hbuf = take(Pm * L.N * d_e * 2);
     } else {
-        L.cntA = L.cntB = L.flags = L.partA = L.partB = 0;
+        L.cntA = L.readyA = L.cntB = L.partA = L.partB = 0;
         L.hbuf = take(Pm * n * d_e * 4);
     }
     L.total = off;
@@ -169,6 +170,10 @@ int blockffn_num_sms(void) { return num_sms_current(); }
 
 void blockffn_debug_skip_flag(int unit) { g_skip_flag.store(unit < 0 ? -1 : unit); }
 
+void blockffn_debug_set_trace(void* device_buffer) {
+    g_trace.store(static_cast<unsigned long long*>(device_buffer));
+}
+
 blockffn_status blockffn_route(const void* x, const void* W_r, const float* b_r,
                                const float* gamma, float eps, int T, int d_h, int E,
                                blockffn_dtype dt, float* gates, void* stream) {
@@ -218,6 +223,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
                                  size_t ws_bytes, void* stream) {
     blockffn_status st = check_shapes(T, d_h, E, d_e, n, dt);
     if (st != BLOCKFFN_OK) return st;
+    if (T == 0) return BLOCKFFN_OK;   // nothing to compute (empty tensors may be NULL)
     const bool routed = gates == nullptr;
     if (routed) {
         if (!W_r || !gamma) return fail(BLOCKFFN_ERR_INVALID_ARG, "no gates: W_r and gamma are required");
@@ -227,7 +233,6 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     } else if (W_r || b_r || gamma) {
         return fail(BLOCKFFN_ERR_INVALID_ARG, "pass either gates or router weights, not both");
     }
-    if (T == 0) return BLOCKFFN_OK;
     if (!x || !W_in || !W_out || !y || !workspace) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(x) || !aligned16(W_in) || !aligned16(W_out) || !aligned16(y) ||
         !aligned16(workspace) || (gates && !aligned16(gates)) || (W_r && !aligned16(W_r)) ||
@@ -268,15 +273,62 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     }
 
     const bool fuse = L.C == 1;
+    static int pairs_cache[64];
+    static std::once_flag pairs_once[64];
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    int npairs = -1;
+    if (fuse && dev_id >= 0 && dev_id < 64) {
+        std::call_once(pairs_once[dev_id], [&]() { pairs_cache[dev_id] = decode_max_pairs(); });
+        npairs = pairs_cache[dev_id];
+        if (npairs > G / 2) npairs = G / 2;
+    }
+    if (fuse && npairs > 0 && 2 * npairs <= 160 && L.KB % 2 == 0) {
+        // one chunk: expert-in split in k-halves over pairs of blocks
+        // (forward_decode.cu)
+        const int Gd = 2 * npairs;
+        CUtensorMap dmaps[3];
+        if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
+            !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
+            !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128))
+            return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+        DcArgs da;
+        da.gates = g;
+        da.y = static_cast<__nv_bfloat16*>(y);
+        da.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
+        da.partB = reinterpret_cast<float*>(ws + L.partB);
+        da.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
+        da.cntB = reinterpret_cast<uint32_t*>(ws + L.cntB);
+        da.ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
+        da.T = T;
+        da.d_h = d_h;
+        da.E = E;
+        da.d_e = d_e;
+        da.n = n;
+        da.N = L.N;
+        da.KB = L.KB;
+        da.RT = L.RT;
+        da.skip_unit = g_skip_flag.load();
+        da.wait_ns = g_wait_ns.load();
+        da.trace = g_trace.load();
+        static std::atomic<int> coop_ok{1};
+        if (coop_ok.load()) {
+            e = launch_forward_decode(da, dmaps, Gd, s, true);
+            if (e == cudaSuccess) return BLOCKFFN_OK;
+            cudaGetLastError();
+            coop_ok.store(0);   // clusters with a cooperative launch are not available here
+        }
+        e = launch_forward_decode(da, dmaps, Gd, s, false);
+        return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "single-chunk forward launch");
+    }
     if (!fuse) {
         e = launch_chunk_union_plan(g, T, E, n, counts, idx, tmask, offsets, pair_ce, y, d_h, 2, s);
         if (e != cudaSuccess) return cuda_fail(e, "union launch");
     }
-    CUtensorMap maps[4];
+    CUtensorMap maps[3];
     if (!make_map(&maps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
         !make_map(&maps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
-        !make_map(&maps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
-        !make_map(&maps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)L.Pmax * L.N, (uint32_t)L.N))
+        !make_map(&maps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128))
         return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     TcArgs a;
     a.gates = g;
@@ -288,8 +340,10 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.partA = reinterpret_cast<float*>(ws + L.partA);
     a.partB = reinterpret_cast<float*>(ws + L.partB);
     a.cntA = reinterpret_cast<uint32_t*>(ws + L.cntA);
+    a.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
     a.cntB = reinterpret_cast<uint32_t*>(ws + L.cntB);
-    a.flags = reinterpret_cast<uint32_t*>(ws + L.flags);
+    a.cnt_a_len = L.Pmax * L.MT;
+    a.cnt_b_len = (long long)L.C * L.RT;
     a.ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
     a.y = static_cast<__nv_bfloat16*>(y);
     a.T = T;
@@ -306,6 +360,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.fuse_union = fuse ? 1 : 0;
     a.wait_ns = g_wait_ns.load();
     a.skip_flag_unit = g_skip_flag.load();
+    a.trace = g_trace.load();
     e = launch_forward_tc(a, maps, G, s);
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "tensor-core forward launch");
 }

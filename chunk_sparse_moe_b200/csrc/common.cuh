@@ -29,6 +29,7 @@ enum : int32_t {
     kWaitFlag = 6,       // activation loader waiting for another block's result
     kWaitDrain = 7,      // teardown waiting for its own copies in flight
     kWaitMmaDone = 8,    // teardown waiting for the last MMAs
+    kWaitPeers = 9,      // a split unit's block waiting for the other contributors
 };
 
 // Control block at offset 0 of every forward workspace (256 bytes reserved).
@@ -63,6 +64,23 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_
     }
 }
 
+// Same, acquiring at cluster scope (for barriers that blocks of the cluster
+// arrive on remotely).
+__device__ __forceinline__ bool wait_bar_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                 volatile int* abort, Ctl* ctl, int32_t detail) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            record_error(ctl, kErrTimeout, detail);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
 // Same, without the abort short-cut: used at teardown to let copies land.
 __device__ __forceinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity,
                                                uint64_t limit_ns, Ctl* ctl) {
@@ -77,17 +95,19 @@ __device__ __forceinline__ bool wait_bar_drain(uint64_t* bar, uint32_t parity,
     }
 }
 
-// Spin until *flag == want (acquire), bounded.
-__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t want, uint64_t limit_ns,
-                                          volatile int* abort, Ctl* ctl) {
-    if (ld_acquire_gpu(flag) == want) return true;
+// Spin until the counter reaches want (acquire), bounded.  detail tells which
+// wait this is when it runs out.
+__device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t want, uint64_t limit_ns,
+                                           volatile int* abort, Ctl* ctl,
+                                           int32_t detail = kWaitFlag) {
+    if (ld_acquire_gpu(ctr) >= want) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        __nanosleep(64);
-        if (ld_acquire_gpu(flag) == want) return true;
+        __nanosleep(32);
+        if (ld_acquire_gpu(ctr) >= want) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
-            record_error(ctl, kErrTimeout, kWaitFlag);
+            record_error(ctl, kErrTimeout, detail);
             *abort = 1;
             return false;
         }

@@ -38,9 +38,12 @@ struct TcArgs {
     __nv_bfloat16* hbuf;      // [C*E*N, d_e] gated activations of every pair
     float* partA;             // [grid][2][N*128] split-K partial sums (expert-in GEMM)
     float* partB;             // [grid][2][N*128] split-expert partial sums (expert-out GEMM)
-    uint32_t* cntA;           // [C*E*MT] arrival counters
-    uint32_t* cntB;           // [C*RT]
-    uint32_t* flags;          // [C*E*MT] "gated activation ready" stamps
+    // counters, two sets chosen by launch parity (each launch zeroes the other set)
+    uint32_t* cntA;           // [2][cnt_a_len] blocks that published an expert-in partial
+    uint32_t* readyA;         // [2][cnt_a_len] blocks whose rows of h' are written
+    uint32_t* cntB;           // [2][cnt_b_len] blocks that published an expert-out partial
+    long long cnt_a_len;      // C*E*MT: expert-in units
+    long long cnt_b_len;      // C*RT: expert-out units
     Ctl* ctl;
     __nv_bfloat16* y;         // [T, d_h]
     int T, d_h, E, d_e, n, N, C;
@@ -49,12 +52,37 @@ struct TcArgs {
     int RT;    // d_h / 128: 128-row tiles of y
     int KBe;   // d_e / 64: k-blocks of one expert in the expert-out GEMM
     int fuse_union;   // 1 when C == 1: each block forms the union itself from gates
-    int skip_flag_unit;   // test support: never publish this A unit's flag (-1: off)
+    int skip_flag_unit;   // test support: unit whose h' is never announced ready (-1: off)
+    unsigned long long* trace;   // optional [grid][16] globaltimer stamps (nullptr: off)
     unsigned long long wait_ns;
 };
 
-// maps: x, W_in, W_out, hbuf (2-D, bf16, 128-byte swizzle, boxes {64,N},{64,128},{64,128},{64,N})
+// maps: x, W_in, W_out (2-D, bf16, 128-byte swizzle, boxes {64,N}, {64,128}, {64,128})
 cudaError_t launch_forward_tc(const TcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s);
 size_t forward_tc_smem_bytes();
+
+// Arguments of the single-chunk forward (see forward_decode.cu): expert-in
+// units are (union expert, 128-row tile of W_in) split along K over a pair of
+// blocks (a cluster of 2); expert-out row tiles are split over blocks and
+// reduced in two passes.
+struct DcArgs {
+    const float* gates;       // [T, E], T <= n
+    __nv_bfloat16* y;         // [T, d_h]
+    __nv_bfloat16* hbuf;      // [E slots][N][d_e] gated activations h'
+    float* partB;             // [grid][2][N*128] expert-out partial tiles
+    uint32_t* readyA;         // [2][E] quarters of an expert slot written, by launch parity
+    uint32_t* cntB;           // [2][RT] expert-out partials published, by launch parity
+    Ctl* ctl;
+    int T, d_h, E, d_e, n, N;
+    int KB;    // d_h / 64
+    int RT;    // d_h / 128
+    int skip_unit;            // test support: expert-in half never counted in (-1: off)
+    unsigned long long wait_ns;
+    unsigned long long* trace;   // optional [grid][32] globaltimer stamps
+};
+cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s,
+                                  bool cooperative);
+size_t forward_decode_smem_bytes();
+int decode_max_pairs();
 
 }  // namespace bffn

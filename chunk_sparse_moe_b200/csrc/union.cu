@@ -5,9 +5,10 @@
 // processes n consecutive tokens at once and computes only the union of the
 // experts any of them activates.
 //
-// One warp per chunk.  Lane l owns experts l, l+32, ...; for each token of the
-// chunk it reads one gate per owned expert (a coalesced 128-byte row segment per
-// token) and ORs the token's active bit into a 32-bit token mask.  A ballot over
+// One warp per chunk.  Lane l owns experts l, l+32, ...; it reads its expert's
+// gate for every token of the chunk (for each token the warp reads a coalesced
+// 128-byte row segment; all loads are in flight together) and ORs the tokens'
+// active bits into a 32-bit token mask.  A ballot over
 // the lanes' "any token active" bits then compacts the active experts of each
 // 32-expert group in ascending order (prefix popcount of the ballot).
 #include <cuda_bf16.h>
@@ -28,14 +29,15 @@ __device__ __forceinline__ void union_one_chunk(const float* __restrict__ gates,
     const int nt = min(n, T - t0);
     for (int g0 = 0; g0 < E; g0 += 32) {
         const int e = g0 + lane;
+        // all n loads of the lane are issued before the first use
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            v[j] = (e < E && j < nt) ? __ldg(gates + (size_t)(t0 + j) * E + e) : 0.f;
         uint32_t bits = 0u;
-        if (e < E) {
-            for (int j = 0; j < nt; ++j) {
-                const float v = __ldg(gates + (size_t)(t0 + j) * E + e);
-                bits |= (v != 0.0f ? 1u : 0u) << j;
-            }
-            tmask[(size_t)c * E + e] = bits;
-        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) bits |= (v[j] != 0.0f ? 1u : 0u) << j;
+        if (e < E) tmask[(size_t)c * E + e] = bits;
         const uint32_t bal = __ballot_sync(0xffffffffu, bits != 0u);
         if (bits != 0u) idx[(size_t)c * E + base + __popc(bal & ((1u << lane) - 1u))] = e;
         base += __popc(bal);

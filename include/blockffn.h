@@ -167,13 +167,29 @@ void blockffn_set_wait_limit_ns(uint64_t ns);
 
 /*
  * blockffn_debug_skip_flag -- failure-detection test support.  For later forward
- * launches (bf16 path), the thread block that finishes expert-in unit `unit`
- * (the unit index is pair * (d_e / 128) + m-tile) writes its activations but
- * never publishes the flag that says so; the expert-out tiles that need them
- * then wait until the bounded-wait limit runs out, and the launch records
- * BLOCKFFN_ERR_TIMEOUT in the workspace.  -1 (the default) turns it off.
+ * launches (bf16 path), the thread blocks that finish expert-in unit `unit`
+ * (the unit index is pair * (d_e / 128) + m-tile) write its activations but never
+ * count them as ready; the expert-out tiles that need them then wait until the
+ * bounded-wait limit runs out, and the launch records BLOCKFFN_ERR_TIMEOUT in the
+ * workspace.  -1 (the default) turns it off.
  */
 void blockffn_debug_skip_flag(int unit);
+
+/*
+ * blockffn_debug_set_trace -- timeline tracing of later bf16 forward launches.
+ * device_buffer (device memory, zeroed by the caller, blockffn_num_sms() * 32
+ * uint64 entries) receives, per thread block, globaltimer stamps in nanoseconds:
+ * 0 start, 1 prologue done, 2 first weight load issued, 3 last load issued,
+ * 4 first tile landed, 5 last expert-in accumulator committed, 6 first
+ * accumulator drained, 7 last expert-in unit finished, 8 first and 9 last
+ * activation flag seen, 10 last accumulator committed, 11 last unit finished,
+ * 12 teardown, 13 end; for the block's first expert-in (A) and expert-out (B)
+ * unit: 14/21 partial written, 15/22 arrival counted, 16/23 partials summed,
+ * 17 activations published; 18 gates loaded, 19 control word loaded, 20 TMEM
+ * allocated, 24 first activation tile copied, 25 first expert-out MMA issued.
+ * Unset stamps stay 0.  NULL (the default) turns tracing off.
+ */
+void blockffn_debug_set_trace(void* device_buffer);
 
 /*
  * blockffn_num_sms -- streaming multiprocessors of the current device (the grid

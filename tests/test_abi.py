@@ -68,6 +68,7 @@ def test_forward_rejects_bad_shapes_on_host(lib, T, d_h, E, d_e, n, dt):
 
 def test_forward_gating_source_is_exclusive(lib):
     L = lib.lib
+    # (T = 32 > 0: with T = 0 the call is a no-op before this check)
     # gates and router weights together
     st = L.blockffn_forward(16, 16, 16, None, None, 0.0, 16, 16, 32, 2048, 64, 128, 32, 1, 16, 16,
                             1 << 30, None)

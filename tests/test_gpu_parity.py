@@ -68,8 +68,12 @@ def _check_route(bffn, w):
     logits, g_ref = oracle.route(w.x, w.W_r, w.gamma, w.eps, b_r=w.b_r)
     band = router_mask_band(w)
     sure = np.abs(logits) > band
+    # outside the worst-case fp32 rounding band of the logit the mask is bit-exact
     assert np.array_equal((g != 0)[sure], (g_ref != 0)[sure]), "gate-zero mask differs"
-    assert np.sum(~sure) <= max(1, int(1e-3 * g.size)), "too many logits inside the band"
+    # inside it either bit is a correct rounding of the fp32 sum; typical errors are
+    # ~1000x below the worst-case band, so flips stay rare
+    flips = int(np.sum((g != 0)[~sure] != (g_ref != 0)[~sure]))
+    assert flips <= max(3, int(1e-5 * g.size)), f"{flips} mask flips inside the band"
     # values: fp32 accumulation and normalisation
     both = (g != 0) & (g_ref != 0)
     err = np.max(np.abs(g - g_ref)[both]) if np.any(both) else 0.0
