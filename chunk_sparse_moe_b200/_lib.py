@@ -39,6 +39,8 @@ SIGNATURES = {
                                  c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                  c_void_p, c_void_p, c_size_t, c_void_p]),
     "blockffn_get_device_status": (c_int, [c_void_p, c_void_p, c_int32_p]),
+    "blockffn_forward_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                                         c_int, c_int, c_int, c_void_p, c_void_p]),
     "blockffn_set_wait_limit_ns": (None, [c_uint64]),
     "blockffn_num_sms": (c_int, []),
     "blockffn_debug_skip_flag": (None, [c_int]),

@@ -365,6 +365,109 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "tensor-core forward launch");
 }
 
+// ------------------------------------------------------------------------
+// blockffn_forward_noalloc: the single-chunk forward without a caller-provided
+// workspace.  Its scratch is the file-scope device array below, which every GPU
+// that loads this library holds until the process exits.  Host code must not
+// pass g_noalloc_scratch itself to a kernel (on the host it names a host-side
+// stand-in); the device address comes from cudaGetSymbolAddress, taken once per
+// device on the first call with that device current.
+// ------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* noalloc_scratch_ptr(int dev, cudaError_t* err) {
+    static void* ptrs[64];
+    static cudaError_t errs[64];
+    static std::once_flag once[64];
+    std::call_once(once[dev], [dev]() {
+        void* p = nullptr;
+        errs[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // the current device is `dev`
+        ptrs[dev] = errs[dev] == cudaSuccess ? p : nullptr;
+    });
+    *err = errs[dev];
+    return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, const void* W_in,
+                                         const void* W_out, int T, int d_h, int E, int d_e, int n,
+                                         void* y, void* stream) {
+    blockffn_status st = check_shapes(T, d_h, E, d_e, n, BLOCKFFN_BF16);
+    if (st != BLOCKFFN_OK) return st;
+    if (T > n) return fail(BLOCKFFN_ERR_UNSUPPORTED, "no-allocation forward: one chunk only (T = %d > n = %d)", T, n);
+    if (T == 0) return BLOCKFFN_OK;
+    if (!x || !gates || !W_in || !W_out || !y) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(gates) || !aligned16(W_in) || !aligned16(W_out) || !aligned16(y))
+        return fail(BLOCKFFN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return fail(BLOCKFFN_ERR_CUDA, "no current CUDA device");
+    const int G = num_sms_current();
+    static int pairs_cache[64];
+    static std::once_flag pairs_once[64];
+    std::call_once(pairs_once[dev], [&]() { pairs_cache[dev] = decode_max_pairs(); });
+    int npairs = pairs_cache[dev];
+    if (npairs > G / 2) npairs = G / 2;
+    if (npairs <= 0 || 2 * npairs > 160 || (d_h / 64) % 2 != 0)
+        return fail(BLOCKFFN_ERR_UNSUPPORTED, "no-allocation forward: single-chunk kernel unavailable here");
+    const int Gd = 2 * npairs;
+    const int N = n <= 16 ? 16 : 32;
+    const int RT = d_h / 128;
+    // scratch layout: control block, readiness and arrival counters (the part
+    // that must start at zero), then h' and the expert-out partial tiles
+    const size_t off_ready = 256;
+    const size_t off_cntB = align_up(off_ready + 2 * (size_t)E * 4, 256);
+    const size_t zero_bytes = align_up(off_cntB + 2 * (size_t)RT * 4, 256);
+    const size_t off_h = zero_bytes;
+    const size_t off_part = align_up(off_h + (size_t)E * N * d_e * 2, 256);
+    const size_t need = off_part + (size_t)Gd * 2 * N * 128 * 4;
+    if (need > kNoAllocScratchBytes)
+        return fail(BLOCKFFN_ERR_UNSUPPORTED,
+                    "no-allocation forward: these shapes need %zu bytes of scratch, more than the %zu "
+                    "reserved (E * d_e too large)", need, kNoAllocScratchBytes);
+    cudaError_t e = cudaSuccess;
+    char* scratch = static_cast<char*>(noalloc_scratch_ptr(dev, &e));
+    if (scratch == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // every call starts from a clean control block and counters
+    e = cudaMemsetAsync(scratch, 0, zero_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "no-allocation scratch clear");
+    CUtensorMap dmaps[3];
+    if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)N) ||
+        !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
+        !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128))
+        return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    DcArgs da;
+    da.gates = gates;
+    da.y = static_cast<__nv_bfloat16*>(y);
+    da.hbuf = reinterpret_cast<__nv_bfloat16*>(scratch + off_h);
+    da.partB = reinterpret_cast<float*>(scratch + off_part);
+    da.readyA = reinterpret_cast<uint32_t*>(scratch + off_ready);
+    da.cntB = reinterpret_cast<uint32_t*>(scratch + off_cntB);
+    da.ctl = reinterpret_cast<Ctl*>(scratch);
+    da.T = T;
+    da.d_h = d_h;
+    da.E = E;
+    da.d_e = d_e;
+    da.n = n;
+    da.N = N;
+    da.KB = d_h / 64;
+    da.RT = RT;
+    da.skip_unit = -1;
+    da.wait_ns = g_wait_ns.load();
+    da.trace = nullptr;
+    e = launch_forward_decode(da, dmaps, Gd, s, false);
+    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "no-allocation forward launch");
+}
+
 blockffn_status blockffn_get_device_status(const void* workspace, void* stream, int32_t* detail) {
     if (!workspace) return fail(BLOCKFFN_ERR_INVALID_ARG, "null workspace");
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -148,6 +148,34 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
                                  void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * blockffn_forward_noalloc -- the same layer output as blockffn_forward for ONE
+ * chunk with injected gates (T <= n, bf16), for callers that cannot allocate
+ * device memory: code running where cudaMalloc is not allowed or not wanted,
+ * such as a runtime that plans every device byte ahead of time, a caller inside
+ * a region that must not synchronize the device (cudaMalloc can), or a plug-in
+ * that receives only input and output buffers from its host.  No counterpart in
+ * the paper: this is a calling convention of this library.
+ *
+ * Arguments as in blockffn_forward (x [T, d_h], gates [T, E] fp32, W_in, W_out,
+ * y [T, d_h], device pointers owned by the caller); there is no workspace.  The
+ * scratch is a fixed 8 MiB device array inside the library, which every GPU that
+ * loads the library holds until the process exits.  Shapes whose scratch would
+ * exceed it (roughly E * d_e * 64 bytes plus 32 KB per SM) are rejected with
+ * BLOCKFFN_ERR_UNSUPPORTED; so are T > n and non-bf16 data.  Nothing is
+ * allocated: no cudaMalloc, cudaFree or allocating library call.
+ * The first call on a device looks up the scratch's device address (with that
+ * device current); make that first call before capturing any CUDA graph.  Every
+ * call clears the scratch's counters on `stream` and then launches the forward.
+ * All calls share the one scratch array and it keeps the last call's contents:
+ * calls that can overlap on the GPU (different streams, or concurrent host
+ * threads) race and must not be issued.  Device-side timeouts are not reported
+ * back (there is no workspace to read); use blockffn_forward for that.
+ */
+blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, const void* W_in,
+                                         const void* W_out, int T, int d_h, int E, int d_e, int n,
+                                         void* y, void* stream);
+
+/*
  * blockffn_get_device_status -- synchronize stream, then read the device status
  * word of a workspace: BLOCKFFN_OK, or the first device-side error recorded
  * (BLOCKFFN_ERR_TIMEOUT, BLOCKFFN_ERR_WORKSPACE).  detail (may be NULL) receives
