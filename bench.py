@@ -48,9 +48,11 @@ R_COPIES = 8
 L2_BYTES = 126 * 1024 * 1024
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the forward kernel,
-# from the ncu capture summarised in profiles/ (None until captured for the
-# current kernel).
-TRAFFIC_BYTES_PER_LAUNCH = None
+# from the ncu capture summarised in profiles/union_expert_decode_chunk32.md
+# (mean of the two captured launches; their algorithmic bytes were 30.68 and
+# 36.97 MB, the traffic 30.67 and 36.96 MB).  None when the kernel has changed
+# since the capture.
+TRAFFIC_BYTES_PER_LAUNCH = (30.670080e6 + 2560 + 36.961280e6 + 2304) / 2
 
 
 def peaks():
@@ -405,7 +407,7 @@ def main():
                          "unit": "GB/s", "frac": achieved_gbs / hbm_peak,
                          "traffic": TRAFFIC_BYTES_PER_LAUNCH,
                          "peak_kind": peak_kind,
-                         "kernel": "union_expert_forward_tc",
+                         "kernel": "union_expert_decode",
                          "kernel_us": kernel_ms * 1e3,
                          "algorithmic_bytes_per_launch": mean_bytes,
                          "step_gbs": step_gbs,

@@ -311,13 +311,8 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.skip_unit = g_skip_flag.load();
         da.wait_ns = g_wait_ns.load();
         da.trace = g_trace.load();
-        static std::atomic<int> coop_ok{1};
-        if (coop_ok.load()) {
-            e = launch_forward_decode(da, dmaps, Gd, s, true);
-            if (e == cudaSuccess) return BLOCKFFN_OK;
-            cudaGetLastError();
-            coop_ok.store(0);   // clusters with a cooperative launch are not available here
-        }
+        // A cluster launch cannot also be cooperative; the grid is sized to the
+        // pairs that can be resident at once, and every wait is bounded.
         e = launch_forward_decode(da, dmaps, Gd, s, false);
         return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "single-chunk forward launch");
     }
