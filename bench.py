@@ -48,11 +48,9 @@ R_COPIES = 8
 L2_BYTES = 126 * 1024 * 1024
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of the forward kernel,
-# from the ncu capture summarised in profiles/union_expert_decode_chunk32.md
-# (mean of the two captured launches; their algorithmic bytes were 30.68 and
-# 36.97 MB, the traffic 30.67 and 36.96 MB).  None when the kernel has changed
-# since the capture.
-TRAFFIC_BYTES_PER_LAUNCH = (30.670080e6 + 2560 + 36.961280e6 + 2304) / 2
+# from the ncu capture summarised in profiles/union_expert_decode_chunk32.md.
+# None when the kernel has changed since the capture.
+TRAFFIC_BYTES_PER_LAUNCH = None
 
 
 def peaks():

@@ -66,10 +66,10 @@ def debug_skip_flag(unit: int) -> None:
 
 
 def debug_set_trace(buf: Optional[torch.Tensor]) -> None:
-    """Attach (or detach with None) a zeroed int64 CUDA tensor of num_sms()*32
+    """Attach (or detach with None) a zeroed int64 CUDA tensor of num_sms()*64
     entries that later bf16 forward launches fill with per-block timestamps."""
-    if buf is not None and (buf.dtype != torch.int64 or buf.numel() < 32 * num_sms()):
-        raise ValueError("trace buffer: int64 tensor of at least num_sms()*32 entries")
+    if buf is not None and (buf.dtype != torch.int64 or buf.numel() < 64 * num_sms()):
+        raise ValueError("trace buffer: int64 tensor of at least num_sms()*64 entries")
     lib.blockffn_debug_set_trace(None if buf is None else _ptr(buf))
 
 

@@ -8,6 +8,7 @@
 
 #include <atomic>
 #include <cstdarg>
+#include <cstddef>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -80,7 +81,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 }
 
 struct Layout {
-    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, readyA, cntB, partA, partB, hbuf;
+    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, readyA, cntB, partA, partB, partD, hbuf;
     size_t total;
     int C, N, MT, RT, KB, KBe;
     long long Pmax;
@@ -118,8 +119,11 @@ bool make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         L.partA = take((size_t)G * 2 * L.N * 128 * 4);
         L.partB = take((size_t)G * 2 * L.N * 128 * 4);
         L.hbuf = take(Pm * L.N * d_e * 2);
+        // single-chunk kernel: tagged expert-out partials, apart from the
+        // multi-chunk kernel's plain ones so that no stale word can look tagged
+        L.partD = C == 1 ? take((size_t)G * 2 * L.N * 128 * 8) : 0;
     } else {
-        L.cntA = L.readyA = L.cntB = L.partA = L.partB = 0;
+        L.cntA = L.readyA = L.cntB = L.partA = L.partB = L.partD = 0;
         L.hbuf = take(Pm * n * d_e * 4);
     }
     L.total = off;
@@ -287,18 +291,18 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         // one chunk: expert-in split in k-halves over pairs of blocks
         // (forward_decode.cu)
         const int Gd = 2 * npairs;
-        CUtensorMap dmaps[3];
+        CUtensorMap dmaps[4];
         if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
             !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
-            !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128))
+            !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
+            !make_map(&dmaps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)E * L.N, (uint32_t)L.N))
             return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
         DcArgs da;
         da.gates = g;
         da.y = static_cast<__nv_bfloat16*>(y);
         da.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
-        da.partB = reinterpret_cast<float*>(ws + L.partB);
+        da.partD = reinterpret_cast<unsigned long long*>(ws + L.partD);
         da.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
-        da.cntB = reinterpret_cast<uint32_t*>(ws + L.cntB);
         da.ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
         da.T = T;
         da.d_h = d_h;
@@ -372,7 +376,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 void* noalloc_scratch_ptr(int dev, cudaError_t* err) {
@@ -416,14 +420,15 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     const int Gd = 2 * npairs;
     const int N = n <= 16 ? 16 : 32;
     const int RT = d_h / 128;
-    // scratch layout: control block, readiness and arrival counters (the part
-    // that must start at zero), then h' and the expert-out partial tiles
+    // scratch layout: control block and readiness counters (all but the launch
+    // counter start every call at zero), then h' and the tagged expert-out
+    // partials.  The launch counter stays: a partial is valid only when it
+    // carries the current launch's tag, so tags must never repeat.
     const size_t off_ready = 256;
-    const size_t off_cntB = align_up(off_ready + 2 * (size_t)E * 4, 256);
-    const size_t zero_bytes = align_up(off_cntB + 2 * (size_t)RT * 4, 256);
+    const size_t zero_bytes = align_up(off_ready + 2 * (size_t)E * 4, 256);
     const size_t off_h = zero_bytes;
     const size_t off_part = align_up(off_h + (size_t)E * N * d_e * 2, 256);
-    const size_t need = off_part + (size_t)Gd * 2 * N * 128 * 4;
+    const size_t need = off_part + (size_t)Gd * 2 * N * 128 * 8;
     if (need > kNoAllocScratchBytes)
         return fail(BLOCKFFN_ERR_UNSUPPORTED,
                     "no-allocation forward: these shapes need %zu bytes of scratch, more than the %zu "
@@ -432,21 +437,25 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     char* scratch = static_cast<char*>(noalloc_scratch_ptr(dev, &e));
     if (scratch == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // every call starts from a clean control block and counters
-    e = cudaMemsetAsync(scratch, 0, zero_bytes, s);
+    // clean status and counters for every call; the launch counter (Ctl::epoch)
+    // is left as the previous call set it
+    static_assert(offsetof(Ctl, status) == 0 && offsetof(Ctl, detail) == 4 && offsetof(Ctl, epoch) == 8 &&
+                      offsetof(Ctl, done) == 12, "control block layout");
+    e = cudaMemsetAsync(scratch, 0, 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(scratch + 12, 0, zero_bytes - 12, s);
     if (e != cudaSuccess) return cuda_fail(e, "no-allocation scratch clear");
-    CUtensorMap dmaps[3];
+    CUtensorMap dmaps[4];
     if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)N) ||
         !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
-        !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128))
+        !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
+        !make_map(&dmaps[3], scratch + off_h, (uint64_t)d_e, (uint64_t)E * N, (uint32_t)N))
         return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     DcArgs da;
     da.gates = gates;
     da.y = static_cast<__nv_bfloat16*>(y);
     da.hbuf = reinterpret_cast<__nv_bfloat16*>(scratch + off_h);
-    da.partB = reinterpret_cast<float*>(scratch + off_part);
+    da.partD = reinterpret_cast<unsigned long long*>(scratch + off_part);
     da.readyA = reinterpret_cast<uint32_t*>(scratch + off_ready);
-    da.cntB = reinterpret_cast<uint32_t*>(scratch + off_cntB);
     da.ctl = reinterpret_cast<Ctl*>(scratch);
     da.T = T;
     da.d_h = d_h;

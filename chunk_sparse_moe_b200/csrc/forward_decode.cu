@@ -51,11 +51,12 @@ constexpr int kRsNAccB = 4;                  // expert-out accumulators (32 colu
 constexpr int kRsTmemCols = 256;             // 2 x 32 expert-in + 4 x 32 expert-out columns
 constexpr int kRsMaxE = 256;
 constexpr int kRsMaxG = 160;
-constexpr int kRsPartBytes = 32 * 128 * 4;   // one fp32 partial h^T tile [<=32 tokens][128 rows]
+constexpr int kRsPartBytes = 16 * 128 * 4;   // fp32 partial h^T for the peer's half [<=16 tokens][128 rows]
+constexpr int kRsHStageBytes = 16 * 128 * 2; // this block's half of h' [<=16 tokens][128 rows] bf16
 
 struct RsShared {
     uint64_t full_w[kRsStages];   // TMA bytes landed
-    uint64_t full_h[kRsStages];   // 32 arrivals: h' copies landed (B) / nothing to copy (A)
+    uint64_t full_h[kRsStages];   // h' slice landed (B, TMA bytes) / nothing to copy (A, one arrival)
     uint64_t empty[kRsStages];    // MMAs reading the stage are done
     uint64_t accA_full[2];
     uint64_t accA_empty[2];
@@ -64,12 +65,15 @@ struct RsShared {
     uint64_t part_ready;          // 2 arrivals: both blocks of the pair wrote their partial
     uint64_t part_free;           // 1 arrival: the peer finished reading this block's partial
     uint64_t mma_done;
+    uint64_t a_pub;               // 1 arrival: this block's expert-in results are published
     uint32_t tmem_base;
     volatile int abort;
     uint32_t epoch;
     int P;
     int ep_wait[2];
     int ep_ok;
+    uint32_t trace_once;          // trace slots already stamped (first occurrence only)
+    float s_gate[2][32];          // gates of the current expert-in unit's expert, per token
     int s_contrib[kRsMaxG];
     long long s_blo[kRsMaxG + 1];   // first expert-out tile of every block
     int32_t s_pair_e[kRsMaxE];
@@ -81,17 +85,17 @@ enum : int {
     kRtStart = 0, kRtPrologue = 1, kRtFirstLoad = 2, kRtLastLoad = 3, kRtFirstFull = 4,
     kRtLastACommit = 5, kRtADone = 7, kRtFirstFlag = 8, kRtLastFlag = 9, kRtLastCommit = 10,
     kRtLastEpi = 11, kRtEnd = 13, kRtATmem = 14, kRtAPart = 15, kRtAReady = 16, kRtARead = 17,
-    kRtAWritten = 18, kRtBPartial = 21, kRtBArrive = 22, kRtBReduced = 23, kRtFirstBMma = 24, kRtSlots = 32
+    kRtAWritten = 18, kRtBPartial = 21, kRtBReduced = 23, kRtFirstBMma = 24, kRtSlots = 64
 };
 #define RS_TRACE(slot) \
     do { if (a.trace) a.trace[(size_t)blockIdx.x * kRtSlots + (slot)] = globaltimer_ns(); } while (0)
 #define RS_TRACE_ONCE(slot)                                                            \
     do {                                                                               \
-        if (a.trace && a.trace[(size_t)blockIdx.x * kRtSlots + (slot)] == 0ull)        \
+        if (a.trace && !(atomicOr(&sh.trace_once, 1u << (slot)) & (1u << (slot))))     \
             a.trace[(size_t)blockIdx.x * kRtSlots + (slot)] = globaltimer_ns();        \
     } while (0)
 
-__device__ __forceinline__ float rs_swish(float z) { return z / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float rs_swish(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // block holding expert-out tile j: the last i with blo[i] <= j (ranges may be empty)
 __device__ __forceinline__ int rs_owner(const long long* blo, int G, long long j) {
@@ -104,15 +108,52 @@ __device__ __forceinline__ int rs_owner(const long long* blo, int G, long long j
     return lo;
 }
 
+// Position in the ring of pipeline stages: the stage and the parity of its
+// current use, stepped without divisions.
+struct RingPos {
+    int st = 0;
+    uint32_t ph = 0u;
+    __device__ __forceinline__ void advance() {
+        if (++st == kRsStages) {
+            st = 0;
+            ph ^= 1u;
+        }
+    }
+};
+
+// Expert-out tile j = (rt * P + s) * KBe + kb (row tile, expert slot, k-block),
+// stepped without divisions.
+struct BTile {
+    int rt, s, kb;
+    __device__ __forceinline__ void init(long long j, int P, int KBe) {
+        const long long per = (long long)P * KBe;
+        rt = (int)(j / per);
+        const int rem = (int)(j - (long long)rt * per);
+        s = rem / KBe;
+        kb = rem - s * KBe;
+    }
+    __device__ __forceinline__ void advance(int P, int KBe) {
+        if (++kb == KBe) {
+            kb = 0;
+            if (++s == P) {
+                s = 0;
+                ++rt;
+            }
+        }
+    }
+};
+
 template <int N>
 __global__ void __launch_bounds__(kRsThreads, 1)
 union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_win,
-                    const __grid_constant__ CUtensorMap tm_wout, const DcArgs a) {
+                    const __grid_constant__ CUtensorMap tm_wout, const __grid_constant__ CUtensorMap tm_h,
+                    const DcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     float* part = reinterpret_cast<float*>(smem + kRsStages * kRsStageBytes);     // [N][128] fp32
-    RsShared& sh = *reinterpret_cast<RsShared*>(smem + kRsStages * kRsStageBytes + kRsPartBytes);
+    __nv_bfloat16* hstage = reinterpret_cast<__nv_bfloat16*>(smem + kRsStages * kRsStageBytes + kRsPartBytes);
+    RsShared& sh = *reinterpret_cast<RsShared*>(smem + kRsStages * kRsStageBytes + kRsPartBytes + kRsHStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, cta = blockIdx.x;
     const int KBe = a.d_e / 64;     // 64-wide k-blocks of one expert in the expert-out GEMM
@@ -126,7 +167,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         RS_TRACE(kRtStart);
         for (int s = 0; s < kRsStages; ++s) {
             mbar_init(&sh.full_w[s], 1);
-            mbar_init(&sh.full_h[s], 32);
+            mbar_init(&sh.full_h[s], 1);
             mbar_init(&sh.empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -140,6 +181,8 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         mbar_init(&sh.part_ready, 2);
         mbar_init(&sh.part_free, 1);
         mbar_init(&sh.mma_done, 1);
+        mbar_init(&sh.a_pub, 1);
+        sh.trace_once = 0u;
         fence_mbar_init();
         const int32_t st0 = __ldcg(&a.ctl->status);
         const uint32_t ep0 = __ldcg(&a.ctl->epoch);
@@ -148,6 +191,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_win);
         prefetch_tmap(&tm_wout);
+        prefetch_tmap(&tm_h);
     }
     if (warp == 2) {
         tmem_alloc(&sh.tmem_base, kRsTmemCols);
@@ -180,37 +224,12 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 base += __popc(bal);
             }
             if (lane == 0) sh.P = base;
-            // Expert-out tile ranges, weighted so that every block moves about the
-            // same number of weight bytes (in tiles of 16 KB: an A k-tile or an
-            // expert-out tile).  Pair c has VA/#pairs or one more A units, each
-            // KB/2 k-tiles per block; a block's capacity is what the target leaves
-            // (target = ceil(total / blocks), so the capacities cover all NB tiles);
-            // a warp scan turns them into range starts, clipped at NB.
-            const long long VA = (long long)base * (a.d_e / 128);
+            // Expert-out tile ranges: an even split over all blocks.  The expert-out
+            // MMAs all run after the h' hand-off, so it is their count per block
+            // that sets the length of that phase; the expert-in blocks load their
+            // share after publishing h' (their weights were sent towards L2 early).
             const long long NB = (long long)a.RT * base * KBe;
-            const long long npairs = G / 2;
-            const long long total = VA * a.KB + NB;
-            const long long target = (total + G - 1) / G;
-            const long long q_ua = VA / npairs, r_ua = VA % npairs;
-            long long run = 0;
-            for (int b0 = 0; b0 < G; b0 += 32) {
-                const int i = b0 + lane;
-                long long cap = 0;
-                if (i < G) {
-                    const long long nAi = q_ua + ((i >> 1) < r_ua ? 1 : 0);
-                    cap = target - nAi * (a.KB / 2);
-                    if (cap < 0) cap = 0;
-                }
-                long long incl = cap;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const long long t = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += t;
-                }
-                // the capacities add up to at least NB; ranges stop at NB
-                if (i < G) sh.s_blo[i] = min(NB, run + incl - cap);
-                run += __shfl_sync(0xffffffffu, incl, 31);
-            }
+            for (int i = lane; i < G; i += 32) sh.s_blo[i] = NB * i / G;
             if (lane == 0) sh.s_blo[G] = NB;
         }
     }
@@ -224,7 +243,6 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     const int P = sh.P;
     const int par = (int)(sh.epoch & 1u);
     uint32_t* const readyA = a.readyA + (size_t)par * a.E;
-    uint32_t* const cntB = a.cntB + (size_t)par * a.RT;
     const int VA = P * MT;                                          // A units (expert, 128-row tile)
     const int nA = VA / NCL + (pr < VA % NCL ? 1 : 0);               // A units of this pair
     const long long bLo = sh.s_blo[cta], bHi = sh.s_blo[cta + 1];
@@ -246,49 +264,55 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             const uint64_t pol_stream = policy_evict_first();
             const uint64_t pol_keep = policy_evict_last();
             long long i = 0;
+            RingPos rp;
             bool stop = false;
             for (int ua = 0; ua < nA && !stop; ++ua) {
                 const int v = pr + ua * NCL;
                 const int e = sh.s_pair_e[v / MT], mt = v % MT;
-                for (int t = 0; t < KBh; ++t, ++i) {
+                for (int t = 0; t < KBh; ++t, ++i, rp.advance()) {
                     const int kt = hk * KBh + t;
-                    const int st = (int)(i % kRsStages);
-                    if (!wait_bar(&sh.empty[st], (uint32_t)(((i / kRsStages) & 1) ^ 1), limit, &sh.abort, a.ctl,
-                                  kWaitEmpty)) {
+                    if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
                         stop = true;
                         break;
                     }
-                    uint8_t* w = smem + st * kRsStageBytes;
-                    mbar_arrive_expect_tx(&sh.full_w[st], 16384 + N * 128);
-                    tma_load_2d(w, &tm_win, &sh.full_w[st], kt * 64, e * a.d_e + mt * 128, pol_stream);
-                    tma_load_2d(w + 16384, &tm_x, &sh.full_w[st], kt * 64, 0, pol_keep);
+                    uint8_t* w = smem + rp.st * kRsStageBytes;
+                    mbar_arrive_expect_tx(&sh.full_w[rp.st], 16384 + N * 128);
+                    tma_load_2d(w, &tm_win, &sh.full_w[rp.st], kt * 64, e * a.d_e + mt * 128, pol_stream);
+                    tma_load_2d(w + 16384, &tm_x, &sh.full_w[rp.st], kt * 64, 0, pol_keep);
                     if (i == 0) RS_TRACE(kRtFirstLoad);
                 }
             }
-            // expert-out tiles beyond what the ring holds at once: start them
-            // towards L2 now, so they are near when stages free up
+            // Expert-out weights.  A block with expert-in units sends all of its
+            // tiles towards L2 now and loads them into the ring only after its h' is
+            // published: a release waits for the block's bulk loads in flight, and
+            // no expert-out MMA can start before every h' is out anyway.  Other
+            // blocks load at once and prefetch what the ring cannot hold yet.
             {
-                const long long ahead = (long long)nA * KBh + (bHi - bLo) - kRsStages;
-                for (long long j = bHi - (ahead > 0 ? min(ahead, bHi - bLo) : 0); j < bHi; ++j) {
-                    const int rt = (int)(j / per_rt);
-                    const int rem = (int)(j % per_rt);
-                    tma_prefetch_l2_2d(&tm_wout, (rem % KBe) * 64, sh.s_pair_e[rem / KBe] * a.d_h + rt * 128);
+                const long long nB = bHi - bLo;
+                const long long j0 = nA > 0 ? bLo : bHi - min(nB, max(0LL, nB - (long long)kRsStages));
+                if (j0 < bHi) {
+                    BTile bt;
+                    bt.init(j0, P, KBe);
+                    for (long long j = j0; j < bHi; ++j, bt.advance(P, KBe))
+                        tma_prefetch_l2_2d(&tm_wout, bt.kb * 64, sh.s_pair_e[bt.s] * a.d_h + bt.rt * 128);
                 }
-            }
-            for (long long j = bLo; j < bHi && !stop; ++j, ++i) {
-                const int rt = (int)(j / per_rt);
-                const int rem = (int)(j % per_rt);
-                const int e = sh.s_pair_e[rem / KBe], kb = rem % KBe;
-                const int st = (int)(i % kRsStages);
-                if (!wait_bar(&sh.empty[st], (uint32_t)(((i / kRsStages) & 1) ^ 1), limit, &sh.abort, a.ctl,
-                              kWaitEmpty)) {
+                if (nA > 0 && bLo < bHi && !stop &&
+                    !wait_bar(&sh.a_pub, 0u, limit, &sh.abort, a.ctl, kWaitEmpty))
                     stop = true;
-                    break;
+            }
+            if (bLo < bHi) {
+                BTile bt;
+                bt.init(bLo, P, KBe);
+                for (long long j = bLo; j < bHi && !stop; ++j, ++i, rp.advance(), bt.advance(P, KBe)) {
+                    if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
+                        stop = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.full_w[rp.st], 16384);
+                    tma_load_2d(smem + rp.st * kRsStageBytes, &tm_wout, &sh.full_w[rp.st], bt.kb * 64,
+                                sh.s_pair_e[bt.s] * a.d_h + bt.rt * 128, pol_stream);
+                    if (i == 0) RS_TRACE(kRtFirstLoad);
                 }
-                mbar_arrive_expect_tx(&sh.full_w[st], 16384);
-                tma_load_2d(smem + st * kRsStageBytes, &tm_wout, &sh.full_w[st], kb * 64, e * a.d_h + rt * 128,
-                            pol_stream);
-                if (i == 0) RS_TRACE(kRtFirstLoad);
             }
             RS_TRACE(kRtLastLoad);
             for (long long q = i - kRsStages < 0 ? 0 : i - kRsStages; q < i; ++q)
@@ -299,6 +323,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(128, N);     // 128 weight rows x tokens
             long long i = 0;
+            RingPos rp;
             bool stop = sh.abort != 0;
             for (int ua = 0; ua < nA && !stop; ++ua) {
                 const int ab = ua & 1;
@@ -307,11 +332,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem + accA_col + (uint32_t)(ab * 32);
-                for (int t = 0; t < KBh; ++t, ++i) {
-                    const int st = (int)(i % kRsStages);
-                    const uint32_t ph = (uint32_t)((i / kRsStages) & 1);
-                    if (!wait_bar(&sh.full_w[st], ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
-                        !wait_bar(&sh.full_h[st], ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
+                for (int t = 0; t < KBh; ++t, ++i, rp.advance()) {
+                    const int st = rp.st;
+                    if (!wait_bar(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
+                        !wait_bar(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
                         stop = true;
                         break;
                     }
@@ -342,17 +366,15 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem + accB_col + (uint32_t)(ab * 32);
-                for (long long jj = j; jj < shi; ++jj, ++i) {
-                    const int st = (int)(i % kRsStages);
-                    const uint32_t ph = (uint32_t)((i / kRsStages) & 1);
-                    if (!wait_bar(&sh.full_w[st], ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
-                        !wait_bar(&sh.full_h[st], ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
+                for (long long jj = j; jj < shi; ++jj, ++i, rp.advance()) {
+                    const int st = rp.st;
+                    if (!wait_bar(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
+                        !wait_bar(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
                         stop = true;
                         break;
                     }
                     tc_fence_after();
-                    fence_proxy_async_smem();   // h' slices were written by cp.async
-                    RS_TRACE_ONCE(kRtFirstBMma);
+                    if (jj == bLo) RS_TRACE(kRtFirstBMma);
                     const uint32_t wb = smem_u32(smem + st * kRsStageBytes);
                     const uint32_t hb = wb + 16384;
 #pragma unroll
@@ -370,56 +392,69 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             umma_commit(&sh.mma_done);
         }
     } else if (warp == 2) {
-        // ------------------------------------------------ h' loader (whole warp) --
-        // A stages carry no h': the 32 lanes just arrive.  An expert-out tile of
-        // expert slot s waits (lane 0, bounded) until both halves of every 128-row
-        // tile of s are counted in, then every lane copies its 16-byte pieces of the [N x 64]
-        // slice with cp.async; each lane's arrival fires when its copies land.
-        constexpr int kPieces = N * 8 / 32;
-        long long i = 0;
-        bool stop = sh.abort != 0;
-        uint32_t seen[kRsMaxE / 32];
-#pragma unroll
-        for (int w = 0; w < kRsMaxE / 32; ++w) seen[w] = 0u;
+        // ------------------------------------------------------- h' loader --
+        // A stages carry no h': lane 0 just arrives.  Before the first expert-out
+        // tile the warp waits (bounded) until every expert slot's h' is counted in;
+        // then lane 0 moves each tile's [N x 64] h' slice with one TMA load, which
+        // lands in the same 128-byte-swizzled layout as the weight tile's operand.
         const long long nAt = (long long)nA * KBh;
         const long long total_tiles = nAt + (bHi - bLo);
-        for (; i < total_tiles && !stop; ++i) {
-            const int st = (int)(i % kRsStages);
-            int ok = 1;
-            if (lane == 0)
-                ok = wait_bar(&sh.empty[st], (uint32_t)(((i / kRsStages) & 1) ^ 1), limit, &sh.abort, a.ctl,
-                              kWaitEmpty) ? 1 : 0;
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            if (i < nAt) {
-                mbar_arrive(&sh.full_h[st]);
-                continue;
+        long long i = 0;
+        RingPos rp;
+        int stop = sh.abort != 0;
+        if (lane == 0) {
+            for (; i < nAt; ++i, rp.advance()) {
+                if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
+                    stop = 1;
+                    break;
+                }
+                mbar_arrive(&sh.full_h[rp.st]);
             }
-            const long long j = bLo + (i - nAt);
-            const int rem = (int)(j % per_rt);
-            const int s = rem / KBe, kb = rem % KBe;
-            // slots already seen complete need no further acquire (lane 0 keeps a
-            // bitmask of them; after its acquire the warp barrier orders the
-            // lanes' copies behind it)
-            if (lane == 0 && !((seen[s >> 5] >> (s & 31)) & 1u)) {
-                ok = wait_count(&readyA[s], (uint32_t)(2 * MT), limit_peer, &sh.abort, a.ctl, kWaitFlag) ? 1 : 0;
-                if (ok) {
-                    seen[s >> 5] |= 1u << (s & 31);
-                    RS_TRACE_ONCE(kRtFirstFlag);
-                    RS_TRACE(kRtLastFlag);
+        }
+        stop = __shfl_sync(0xffffffffu, stop, 0);
+        if (!stop && total_tiles > nAt) {
+            // The expert-in units all finish at about the same time, so one combined
+            // wait costs no more than the slowest slot; each poll round checks 32
+            // slots at once (one acquire load per lane).
+            const uint64_t t0 = globaltimer_ns();
+            bool done = false;
+            while (!done) {
+                bool mine_ok = true;
+                for (int q = lane; q < P; q += 32)
+                    if (ld_acquire_gpu(&readyA[q]) < (uint32_t)(2 * MT)) mine_ok = false;
+                done = __all_sync(0xffffffffu, mine_ok);
+                if (done) break;
+                __nanosleep(64);
+                if (__any_sync(0xffffffffu, sh.abort != 0)) break;
+                if (globaltimer_ns() - t0 > limit_peer) {
+                    if (lane == 0) {
+                        record_error(a.ctl, kErrTimeout, kWaitFlag);
+                        sh.abort = 1;
+                    }
+                    break;
                 }
             }
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const uint4* src = reinterpret_cast<const uint4*>(a.hbuf + (size_t)s * N * a.d_e + (size_t)kb * 64);
-            uint8_t* dst = smem + st * kRsStageBytes + 16384;
-#pragma unroll
-            for (int k = 0; k < kPieces; ++k) {
-                const int c = lane + 32 * k;
-                const int r = c >> 3, c16 = c & 7;
-                cp_async_16(dst + r * 128 + ((c16 ^ (r & 7)) << 4), src + (size_t)r * (a.d_e / 8) + c16);
+            __syncwarp();
+            if (lane == 0 && done) {
+                // the h' stores were made visible to this thread by the acquires; the
+                // async proxy reads them next
+                fence_proxy_async_global();
+                RS_TRACE_ONCE(kRtFirstFlag);
+                RS_TRACE(kRtLastFlag);
+                const uint64_t pol = policy_evict_first();
+                BTile bt;
+                bt.init(bLo, P, KBe);
+                for (; i < total_tiles; ++i, rp.advance(), bt.advance(P, KBe)) {
+                    if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) break;
+                    mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 128));
+                    tma_load_2d(smem + rp.st * kRsStageBytes + 16384, &tm_h, &sh.full_h[rp.st], bt.kb * 64,
+                                bt.s * N, pol);
+                }
+                // no copy into this block's shared memory outlives it
+                for (long long q = i - kRsStages < nAt ? nAt : i - kRsStages; q < i; ++q)
+                    wait_bar_drain(&sh.full_h[q % kRsStages], (uint32_t)((q / kRsStages) & 1), limit, a.ctl);
             }
-            cp_async_mbar_arrive(&sh.full_h[st]);
         }
-        cp_async_wait_all();   // no copy into this block's shared memory outlives it
     } else {
         // --------------------------------------------------------- epilogue --
         const int qd = warp & 3;
@@ -429,7 +464,6 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             // zero the other parity's counters for the next launch
             const int oth = par ^ 1;
             for (int k2 = cta * 128 + et; k2 < a.E; k2 += G * 128) a.readyA[(size_t)oth * a.E + k2] = 0u;
-            for (int k2 = cta * 128 + et; k2 < a.RT; k2 += G * 128) a.cntB[(size_t)oth * a.RT + k2] = 0u;
         }
         bool failed = sh.abort != 0;
         const int nt = min(a.n, a.T);
@@ -444,12 +478,14 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             const uint32_t peer_ready = mapa_shared(smem_u32(&sh.part_ready), peer);
             const uint32_t own_ready = mapa_shared(smem_u32(&sh.part_ready), (uint32_t)hk);
             const uint32_t peer_free = mapa_shared(smem_u32(&sh.part_free), peer);
-            const bool mine = (row >> 6) == hk;             // rows [64*hk, 64*hk + 64) are reduced here
             for (int ua = 0; ua < nA && !failed; ++ua) {
                 const int ab = ua & 1;
                 const int v = pr + ua * NCL;
                 const int s = v / MT, mt = v % MT;
                 const int e = sh.s_pair_e[s];
+                // stage the unit's gates now: the accumulator wait hides their latency,
+                // and the activation loop below then reads shared memory only
+                if (et < 32) sh.s_gate[ab][et] = a.gates[(size_t)min(et, nt - 1) * a.E + e];
                 if (et == 0) {
                     int ok = wait_bar(&sh.accA_full[ab], (uint32_t)((ua >> 1) & 1), limit, &sh.abort, a.ctl,
                                       kWaitAccFull) ? 1 : 0;
@@ -471,19 +507,24 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.accA_empty[ab]);
                 if (et == 0) RS_TRACE_ONCE(kRtATmem);
-                // this block's partial h^T tile: float4 of tokens 4k..4k+3 of a row at k*128 + row
+                // The pair splits the chunk's tokens: this block finishes tokens
+                // [tg, tg + NH) of all 128 rows and the peer the other half.  Each block
+                // hands the peer its partial for the peer's tokens: float4 of the half's
+                // tokens 4k..4k+3 of a row at k*128 + row.
+                constexpr int NH = N / 2;
+                const int tg = hk * NH;
                 {
                     float4* p4 = reinterpret_cast<float4*>(part) + row;
 #pragma unroll
-                    for (int k4 = 0; k4 < N / 4; ++k4)
-                        p4[k4 * 128] = make_float4(__uint_as_float(r[4 * k4]), __uint_as_float(r[4 * k4 + 1]),
-                                                   __uint_as_float(r[4 * k4 + 2]), __uint_as_float(r[4 * k4 + 3]));
-                }
-                // the gates of expert e for this chunk (independent of the peer)
-                const uint32_t bits = sh.s_tmask[e];
-                float gv[N];
+                    for (int k4 = 0; k4 < NH / 4; ++k4) {
+                        float f[4];
 #pragma unroll
-                for (int t = 0; t < N; ++t) gv[t] = __ldg(a.gates + (size_t)min(t, nt - 1) * a.E + e);
+                        for (int u = 0; u < 4; ++u)
+                            f[u] = __uint_as_float(hk ? r[4 * k4 + u] : r[NH + 4 * k4 + u]);
+                        p4[k4 * 128] = make_float4(f[0], f[1], f[2], f[3]);
+                    }
+                }
+                const uint32_t bits = sh.s_tmask[e] >> tg;   // this half's token bits
                 named_bar_sync(1, 128);
                 if (et == 0) {
                     RS_TRACE_ONCE(kRtAPart);
@@ -495,19 +536,20 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 }
                 named_bar_sync(1, 128);
                 if (!sh.ep_ok) { failed = true; break; }
-                float z[N];
-                if (mine) {
-                    // h = (k-half 0) + (k-half 1); two terms, so the order is fixed
-                    float4 pv[N / 4];
+                // h = (k-half 0) + (k-half 1): two terms, and the sum does not depend on
+                // which block of the pair forms it
+                float z[NH];
+                {
+                    float4 pv[NH / 4];
 #pragma unroll
-                    for (int k4 = 0; k4 < N / 4; ++k4)
+                    for (int k4 = 0; k4 < NH / 4; ++k4)
                         pv[k4] = ld_shared_cluster_f4(peer_part + (uint32_t)((k4 * 128 + row) * 16));
 #pragma unroll
-                    for (int k4 = 0; k4 < N / 4; ++k4) {
-                        z[4 * k4] = __uint_as_float(r[4 * k4]) + pv[k4].x;
-                        z[4 * k4 + 1] = __uint_as_float(r[4 * k4 + 1]) + pv[k4].y;
-                        z[4 * k4 + 2] = __uint_as_float(r[4 * k4 + 2]) + pv[k4].z;
-                        z[4 * k4 + 3] = __uint_as_float(r[4 * k4 + 3]) + pv[k4].w;
+                    for (int k4 = 0; k4 < NH / 4; ++k4) {
+                        const float pw[4] = {pv[k4].x, pv[k4].y, pv[k4].z, pv[k4].w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            z[4 * k4 + u] = __uint_as_float(hk ? r[NH + 4 * k4 + u] : r[4 * k4 + u]) + pw[u];
                     }
                 }
                 named_bar_sync(1, 128);
@@ -515,23 +557,49 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     RS_TRACE_ONCE(kRtARead);
                     mbar_arrive_cluster(peer_free);   // done with the peer's partial
                 }
-                if (mine) {
-                    __nv_bfloat16* hrow = a.hbuf + (size_t)s * N * a.d_e + mt * 128 + row;
+                // h' = bit ? g * Swish(h) : 0 (a select, so a masked token gives 0 even if
+                // its h is not finite), staged token-major in shared memory, then written
+                // with 16-byte stores: token t's 128 rows are 256 contiguous bytes
+                {
+                    __nv_bfloat16* stg = hstage + row;
 #pragma unroll
-                    for (int t = 0; t < N; ++t) {
-                        const float hv = ((bits >> t) & 1u) ? gv[t] * rs_swish(z[t]) : 0.f;
-                        hrow[(size_t)t * a.d_e] = __float2bfloat16_rn(hv);
+                    for (int tl = 0; tl < NH; ++tl) {
+                        const float gsw = sh.s_gate[ab][tg + tl] * rs_swish(z[tl]);
+                        stg[tl * 128] = __float2bfloat16_rn(((bits >> tl) & 1u) ? gsw : 0.f);
                     }
                 }
-                __threadfence();
                 named_bar_sync(1, 128);
-                if (et == 0) RS_TRACE_ONCE(kRtAWritten);
-                if (et == 0 && (v * 2 + hk) != a.skip_unit) atomicAdd(&readyA[s], 1u);
+                {
+                    const uint4* src4 = reinterpret_cast<const uint4*>(hstage);
+                    for (int c = et; c < NH * 16; c += 128) {
+                        const int tl = c >> 4, c16 = c & 15;
+                        uint4* dst4 =
+                            reinterpret_cast<uint4*>(a.hbuf + ((size_t)s * N + tg + tl) * a.d_e + mt * 128) + c16;
+                        *dst4 = src4[c];
+                    }
+                }
+                // one release for the whole block: the barrier orders every thread's
+                // stores before thread 0's releasing count
+                named_bar_sync(1, 128);
+                if (et == 0) {
+                    if ((v * 2 + hk) != a.skip_unit) red_release_add_gpu(&readyA[s], 1u);
+                    RS_TRACE_ONCE(kRtAWritten);
+                }
             }
-            if (et == 0) RS_TRACE(kRtADone);
+            if (et == 0) {
+                RS_TRACE(kRtADone);
+                if (nA > 0) mbar_arrive(&sh.a_pub);   // the producer may load expert-out tiles now
+            }
         }
-        // ---- expert-out row tiles: contributors publish partials, then each sums a slice
-        const float* partB = a.partB;
+        // ---- expert-out row tiles.  A row tile whose k-range is split over several
+        // blocks is summed without a flag: every contributor stores its partial as
+        // (launch tag, fp32) pairs with relaxed stores, and the block that sums a
+        // slice of the tile's rows polls those pairs until each carries this
+        // launch's tag, then adds the contributors in block order.
+        const uint32_t tag = sh.epoch + 1u;
+        const unsigned long long tag_hi = (unsigned long long)tag << 32;
+        const size_t slot_pairs = (size_t)(N / 2) * 128;   // 16-byte pairs in one partial slot
+        ulonglong2* const partD = reinterpret_cast<ulonglong2*>(a.partD);
         auto contributors = [&](long long first, long long last, int& q0, int& q1, int& n, int& rank) {
             q0 = rs_owner(sh.s_blo, G, first);
             q1 = rs_owner(sh.s_blo, G, last);
@@ -581,19 +649,13 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     if (t < nt) ycol[(size_t)t * a.d_h] = __float2bfloat16_rn(__uint_as_float(r[t]));
                 if (et == 0) RS_TRACE(kRtLastEpi);
             } else {
+                // pair kp of a row holds tokens 2kp and 2kp+1: [kp][row] x 16 bytes
                 const int myslot = bLo >= first ? 0 : 1;
-                float4* dst = reinterpret_cast<float4*>(a.partB + (size_t)(cta * 2 + myslot) * (N * 128)) + row;
+                ulonglong2* dst = partD + (size_t)(cta * 2 + myslot) * slot_pairs + row;
 #pragma unroll
-                for (int kq = 0; kq < N / 4; ++kq)
-                    dst[kq * 128] = make_float4(__uint_as_float(r[4 * kq]), __uint_as_float(r[4 * kq + 1]),
-                                                __uint_as_float(r[4 * kq + 2]), __uint_as_float(r[4 * kq + 3]));
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (et == 0) {
-                    RS_TRACE_ONCE(kRtBPartial);
-                    atomicAdd(&cntB[rt], 1u);
-                    RS_TRACE_ONCE(kRtBArrive);
-                }
+                for (int kp = 0; kp < N / 2; ++kp)
+                    st_relaxed_v2_b64(dst + kp * 128, tag_hi | r[2 * kp], tag_hi | r[2 * kp + 1]);
+                if (et == 0) RS_TRACE_ONCE(kRtBPartial);
                 if (npend < 2) {
                     pend_first[npend] = first;
                     pend_last[npend] = last;
@@ -603,65 +665,61 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
             j = shi;
         }
-        // second pass: wait for each split row tile's contributors, sum my slice
+        // second pass: sum my slice of each split row tile's rows
         for (int pi = 0; pi < npend && !failed; ++pi) {
             int q0, q1, nc, rank;
             contributors(pend_first[pi], pend_last[pi], q0, q1, nc, rank);
             const int rt = pend_rt[pi];
             if (et == 0) {
-                sh.ep_ok = wait_count(&cntB[rt], (uint32_t)nc, limit_peer, &sh.abort, a.ctl, kWaitPeers) ? 1 : 0;
                 int k2 = 0;
                 for (int qq = q0; qq <= q1 && k2 < kRsMaxG; ++qq)
                     if (sh.s_blo[qq + 1] > sh.s_blo[qq])
                         sh.s_contrib[k2++] = qq * 2 + (sh.s_blo[qq] >= pend_first[pi] ? 0 : 1);
             }
             named_bar_sync(1, 128);
-            if (!sh.ep_ok) { failed = true; break; }
             const int r0 = rank * 128 / nc, r1 = (rank + 1) * 128 / nc, nrows = r1 - r0;
-            const float4* pbase = reinterpret_cast<const float4*>(partB);
-            const int nitems = nrows * (N / 4);
-            for (int base = 0; base < nitems; base += 256) {
-                int rr[2], kq[2];
-                bool on2[2];
+            const int nitems = nrows * (N / 2);
+            const uint64_t t0 = globaltimer_ns();
+            for (int it = et; it < nitems && !failed; it += 128) {
+                const int rr = r0 + it % nrows, kp = it / nrows;
+                float sx = 0.f, sy = 0.f;
+                for (int c0 = 0; c0 < nc && !failed; c0 += 8) {
+                    const ulonglong2* src[8];
+                    ulonglong2 v[8];
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    const int itx = base + m * 128 + et;
-                    on2[m] = itx < nitems;
-                    const int ic = on2[m] ? itx : 0;
-                    rr[m] = r0 + ic % nrows;
-                    kq[m] = ic / nrows;
-                }
-                float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-                for (int c0 = 0; c0 < nc; c0 += 8) {
-                    float4 t4[2][8];
-#pragma unroll
-                    for (int m = 0; m < 2; ++m)
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            t4[m][u] = __ldcg(pbase + (size_t)sh.s_contrib[min(c0 + u, nc - 1)] * (N * 32) +
-                                              kq[m] * 128 + rr[m]);
-#pragma unroll
-                    for (int m = 0; m < 2; ++m)
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            if (c0 + u < nc) {
-                                acc[m].x += t4[m][u].x;
-                                acc[m].y += t4[m][u].y;
-                                acc[m].z += t4[m][u].z;
-                                acc[m].w += t4[m][u].w;
-                            }
-                }
-#pragma unroll
-                for (int m = 0; m < 2; ++m) {
-                    if (!on2[m]) continue;
-                    const float z[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
-                    __nv_bfloat16* ycol = a.y + rt * 128 + rr[m];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int t = 4 * kq[m] + u;
-                        if (t < nt) ycol[(size_t)t * a.d_h] = __float2bfloat16_rn(z[u]);
+                    for (int u = 0; u < 8; ++u) {
+                        src[u] = partD + (size_t)sh.s_contrib[min(c0 + u, nc - 1)] * slot_pairs + kp * 128 + rr;
+                        v[u] = ld_relaxed_v2_b64(src[u]);
                     }
+                    while (true) {   // re-read the pairs that are not this launch's yet (bounded)
+                        bool all = true;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            if ((uint32_t)(v[u].x >> 32) != tag || (uint32_t)(v[u].y >> 32) != tag) {
+                                all = false;
+                                v[u] = ld_relaxed_v2_b64(src[u]);
+                            }
+                        if (all) break;
+                        if (sh.abort) { failed = true; break; }
+                        if (globaltimer_ns() - t0 > limit_peer) {
+                            record_error(a.ctl, kErrTimeout, kWaitPeers);
+                            sh.abort = 1;
+                            failed = true;
+                            break;
+                        }
+                    }
+                    if (failed) break;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (c0 + u < nc) {
+                            sx += __uint_as_float((uint32_t)v[u].x);
+                            sy += __uint_as_float((uint32_t)v[u].y);
+                        }
                 }
+                if (failed) break;
+                __nv_bfloat16* ycol = a.y + rt * 128 + rr;
+                if (2 * kp < nt) ycol[(size_t)(2 * kp) * a.d_h] = __float2bfloat16_rn(sx);
+                if (2 * kp + 1 < nt) ycol[(size_t)(2 * kp + 1) * a.d_h] = __float2bfloat16_rn(sy);
             }
             if (et == 0) RS_TRACE_ONCE(kRtBReduced);
         }
@@ -695,7 +753,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
 }
 
 size_t forward_decode_smem_bytes() {
-    return 1024 + (size_t)kRsStages * kRsStageBytes + kRsPartBytes + sizeof(RsShared);
+    return 1024 + (size_t)kRsStages * kRsStageBytes + kRsPartBytes + kRsHStageBytes + sizeof(RsShared);
 }
 
 template <int N>
@@ -719,7 +777,7 @@ static cudaError_t launch_decode_n(const DcArgs& a, const CUtensorMap* maps, int
     attr[1].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = cooperative ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, union_expert_decode<N>, maps[0], maps[1], maps[2], a);
+    return cudaLaunchKernelEx(&cfg, union_expert_decode<N>, maps[0], maps[1], maps[2], maps[3], a);
 }
 
 cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s,

@@ -69,17 +69,18 @@ struct DcArgs {
     const float* gates;       // [T, E], T <= n
     __nv_bfloat16* y;         // [T, d_h]
     __nv_bfloat16* hbuf;      // [E slots][N][d_e] gated activations h'
-    float* partB;             // [grid][2][N*128] expert-out partial tiles
-    uint32_t* readyA;         // [2][E] quarters of an expert slot written, by launch parity
-    uint32_t* cntB;           // [2][RT] expert-out partials published, by launch parity
+    unsigned long long* partD;  // [grid][2][N/2][128][2] expert-out partials, (launch tag << 32 | fp32 bits)
+    uint32_t* readyA;         // [2][E] halves of an expert slot written, by launch parity
     Ctl* ctl;
     int T, d_h, E, d_e, n, N;
     int KB;    // d_h / 64
     int RT;    // d_h / 128
     int skip_unit;            // test support: expert-in half never counted in (-1: off)
     unsigned long long wait_ns;
-    unsigned long long* trace;   // optional [grid][32] globaltimer stamps
+    unsigned long long* trace;   // optional [grid][64] globaltimer stamps
 };
+// maps: x [T, d_h] (box N rows), W_in [E*d_e, d_h] and W_out [E*d_h, d_e] (box 128
+// rows), h' [E*N, d_e] (box N rows); all boxes 64 wide, 128-byte swizzle
 cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s,
                                   bool cooperative);
 size_t forward_decode_smem_bytes();
