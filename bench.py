@@ -47,10 +47,13 @@ UNIT = "tokens/s"
 R_COPIES = 8
 L2_BYTES = 126 * 1024 * 1024
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of the forward kernel,
-# from the ncu capture summarised in profiles/union_expert_decode_chunk32.md.
-# None when the kernel has changed since the capture.
-TRAFFIC_BYTES_PER_LAUNCH = None
+# DRAM traffic of the forward kernel from the ncu capture summarised in
+# profiles/union_expert_decode_chunk32.md: (algorithmic bytes, dram__bytes_read.sum
+# + dram__bytes_write.sum) of each captured launch.  The capture covers two of the
+# rotating input copies, so the reported per-launch traffic is their
+# traffic / algorithmic ratio times this run's mean algorithmic bytes.  Empty
+# when the kernel has changed since the capture.
+TRAFFIC_CAPTURE = [(30.679e6, 30.624768e6), (36.970e6, 36.915968e6)]
 
 
 def peaks():
@@ -403,7 +406,8 @@ def main():
             },
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak,
                          "unit": "GB/s", "frac": achieved_gbs / hbm_peak,
-                         "traffic": TRAFFIC_BYTES_PER_LAUNCH,
+                         "traffic": (mean_bytes * sum(t for _, t in TRAFFIC_CAPTURE)
+                                     / sum(b for b, _ in TRAFFIC_CAPTURE)) if TRAFFIC_CAPTURE else None,
                          "peak_kind": peak_kind,
                          "kernel": "union_expert_decode",
                          "kernel_us": kernel_ms * 1e3,

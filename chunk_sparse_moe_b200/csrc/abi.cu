@@ -8,7 +8,6 @@
 
 #include <atomic>
 #include <cstdarg>
-#include <cstddef>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -80,8 +79,23 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 tensor [outer, inner], box {box_inner, box_outer}, no swizzle (for
+// tiled stores from a plain row-major shared-memory tile).
+bool make_map_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                    uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Layout {
-    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, readyA, cntB, partA, partB, partD, hbuf;
+    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, readyA, cntB, partA, partB, hbuf;
     size_t total;
     int C, N, MT, RT, KB, KBe;
     long long Pmax;
@@ -119,11 +133,8 @@ bool make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         L.partA = take((size_t)G * 2 * L.N * 128 * 4);
         L.partB = take((size_t)G * 2 * L.N * 128 * 4);
         L.hbuf = take(Pm * L.N * d_e * 2);
-        // single-chunk kernel: tagged expert-out partials, apart from the
-        // multi-chunk kernel's plain ones so that no stale word can look tagged
-        L.partD = C == 1 ? take((size_t)G * 2 * L.N * 128 * 8) : 0;
     } else {
-        L.cntA = L.readyA = L.cntB = L.partA = L.partB = L.partD = 0;
+        L.cntA = L.readyA = L.cntB = L.partA = L.partB = 0;
         L.hbuf = take(Pm * n * d_e * 4);
     }
     L.total = off;
@@ -277,31 +288,31 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     }
 
     const bool fuse = L.C == 1;
-    static int pairs_cache[64];
-    static std::once_flag pairs_once[64];
+    static int clusters_cache[64];
+    static std::once_flag clusters_once[64];
     int dev_id = 0;
     cudaGetDevice(&dev_id);
-    int npairs = -1;
+    int ncl = -1;
     if (fuse && dev_id >= 0 && dev_id < 64) {
-        std::call_once(pairs_once[dev_id], [&]() { pairs_cache[dev_id] = decode_max_pairs(); });
-        npairs = pairs_cache[dev_id];
-        if (npairs > G / 2) npairs = G / 2;
+        std::call_once(clusters_once[dev_id], [&]() { clusters_cache[dev_id] = decode_max_clusters(); });
+        ncl = clusters_cache[dev_id];
+        if (ncl > G / 4) ncl = G / 4;
     }
-    if (fuse && npairs > 0 && 2 * npairs <= 160 && L.KB % 2 == 0) {
-        // one chunk: expert-in split in k-halves over pairs of blocks
-        // (forward_decode.cu)
-        const int Gd = 2 * npairs;
-        CUtensorMap dmaps[4];
+    if (fuse && ncl > 0 && 4 * ncl <= 160 && L.KB % 2 == 0 && E <= 256) {
+        // one chunk: clusters of 4 blocks, expert-in in k-half pairs, expert-out
+        // row tiles summed inside the cluster (forward_decode.cu)
+        const int Gd = 4 * ncl;
+        CUtensorMap dmaps[5];
         if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
             !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
             !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
-            !make_map(&dmaps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)E * L.N, (uint32_t)L.N))
+            !make_map(&dmaps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)E * L.N, (uint32_t)L.N) ||
+            !make_map_plain(&dmaps[4], y, (uint64_t)d_h, (uint64_t)T, 32, (uint32_t)L.N))
             return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
         DcArgs da;
         da.gates = g;
         da.y = static_cast<__nv_bfloat16*>(y);
         da.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
-        da.partD = reinterpret_cast<unsigned long long*>(ws + L.partD);
         da.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
         da.ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
         da.T = T;
@@ -317,7 +328,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.trace = g_trace.load();
         // A cluster launch cannot also be cooperative; the grid is sized to the
         // pairs that can be resident at once, and every wait is bounded.
-        e = launch_forward_decode(da, dmaps, Gd, s, false);
+        e = launch_forward_decode(da, dmaps, Gd, s);
         return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "single-chunk forward launch");
     }
     if (!fuse) {
@@ -376,7 +387,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 void* noalloc_scratch_ptr(int dev, cudaError_t* err) {
@@ -410,25 +421,22 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return fail(BLOCKFFN_ERR_CUDA, "no current CUDA device");
     const int G = num_sms_current();
-    static int pairs_cache[64];
-    static std::once_flag pairs_once[64];
-    std::call_once(pairs_once[dev], [&]() { pairs_cache[dev] = decode_max_pairs(); });
-    int npairs = pairs_cache[dev];
-    if (npairs > G / 2) npairs = G / 2;
-    if (npairs <= 0 || 2 * npairs > 160 || (d_h / 64) % 2 != 0)
+    static int clusters_cache[64];
+    static std::once_flag clusters_once[64];
+    std::call_once(clusters_once[dev], [&]() { clusters_cache[dev] = decode_max_clusters(); });
+    int ncl = clusters_cache[dev];
+    if (ncl > G / 4) ncl = G / 4;
+    if (ncl <= 0 || 4 * ncl > 160 || (d_h / 64) % 2 != 0 || E > 256)
         return fail(BLOCKFFN_ERR_UNSUPPORTED, "no-allocation forward: single-chunk kernel unavailable here");
-    const int Gd = 2 * npairs;
+    const int Gd = 4 * ncl;
     const int N = n <= 16 ? 16 : 32;
     const int RT = d_h / 128;
-    // scratch layout: control block and readiness counters (all but the launch
-    // counter start every call at zero), then h' and the tagged expert-out
-    // partials.  The launch counter stays: a partial is valid only when it
-    // carries the current launch's tag, so tags must never repeat.
+    // scratch layout: control block and readiness counters (the part that must
+    // start at zero), then h'
     const size_t off_ready = 256;
     const size_t zero_bytes = align_up(off_ready + 2 * (size_t)E * 4, 256);
     const size_t off_h = zero_bytes;
-    const size_t off_part = align_up(off_h + (size_t)E * N * d_e * 2, 256);
-    const size_t need = off_part + (size_t)Gd * 2 * N * 128 * 8;
+    const size_t need = off_h + (size_t)E * N * d_e * 2;
     if (need > kNoAllocScratchBytes)
         return fail(BLOCKFFN_ERR_UNSUPPORTED,
                     "no-allocation forward: these shapes need %zu bytes of scratch, more than the %zu "
@@ -437,24 +445,20 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     char* scratch = static_cast<char*>(noalloc_scratch_ptr(dev, &e));
     if (scratch == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // clean status and counters for every call; the launch counter (Ctl::epoch)
-    // is left as the previous call set it
-    static_assert(offsetof(Ctl, status) == 0 && offsetof(Ctl, detail) == 4 && offsetof(Ctl, epoch) == 8 &&
-                      offsetof(Ctl, done) == 12, "control block layout");
-    e = cudaMemsetAsync(scratch, 0, 8, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(scratch + 12, 0, zero_bytes - 12, s);
+    // every call starts from a clean control block and counters
+    e = cudaMemsetAsync(scratch, 0, zero_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "no-allocation scratch clear");
-    CUtensorMap dmaps[4];
+    CUtensorMap dmaps[5];
     if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)N) ||
         !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
         !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
-        !make_map(&dmaps[3], scratch + off_h, (uint64_t)d_e, (uint64_t)E * N, (uint32_t)N))
+        !make_map(&dmaps[3], scratch + off_h, (uint64_t)d_e, (uint64_t)E * N, (uint32_t)N) ||
+        !make_map_plain(&dmaps[4], y, (uint64_t)d_h, (uint64_t)T, 32, (uint32_t)N))
         return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     DcArgs da;
     da.gates = gates;
     da.y = static_cast<__nv_bfloat16*>(y);
     da.hbuf = reinterpret_cast<__nv_bfloat16*>(scratch + off_h);
-    da.partD = reinterpret_cast<unsigned long long*>(scratch + off_part);
     da.readyA = reinterpret_cast<uint32_t*>(scratch + off_ready);
     da.ctl = reinterpret_cast<Ctl*>(scratch);
     da.T = T;
@@ -468,7 +472,7 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     da.skip_unit = -1;
     da.wait_ns = g_wait_ns.load();
     da.trace = nullptr;
-    e = launch_forward_decode(da, dmaps, Gd, s, false);
+    e = launch_forward_decode(da, dmaps, Gd, s);
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "no-allocation forward launch");
 }
 

@@ -9,31 +9,34 @@
 // Losses).
 //
 // One chunk of n <= 32 tokens; every block forms the chunk's union U (ascending)
-// from the gates itself.
+// from the gates itself.  Blocks run in thread-block clusters of 4: ranks 0-1
+// and 2-3 are two k-half pairs.
 //
-// Expert-in (A).  Blocks work in pairs (thread-block clusters of 2).  A unit is
-// one union expert e and one 128-row tile of W_in_e (d_e = 128: the whole
-// expert); pair c takes the units c, c + #pairs, ..., and its block of rank r
-// multiplies the k-half r of W_in_e (tcgen05; weights as the M = 128 operand,
-// the chunk's N tokens as N) into a TMEM accumulator.  The two partial h^T tiles
-// meet in distributed shared memory: rank r adds them for rows [64r, 64r + 64),
-// applies the post-hoc mask, the gate and Swish, writes those rows of h' (bf16)
-// to global memory and counts them in for the expert.  With up to ~74 union
-// experts about one unit per pair, and each block streams its A tiles first;
-// a stage is a 16 KB weight tile and the 4 KB x tile that multiplies it.
-// Expert-out (B).  y^T = sum_e W_out_e h'_e^T with W_out_e's 128-row tiles as
-// the M operand and the tokens as N.  Tiles (row tile, expert, 64-wide k-block)
-// are cut into contiguous ranges, one per block, sized so every block moves the
-// same number of weight bytes counting its A work.  A tile waits (bounded) until
-// all quarters of its expert are counted in, then its h' slice is copied into
-// the stage with cp.async.  A row tile split across blocks is finished in two
-// passes: every contributor publishes its partial tile, then each sums one
-// slice of rows over all the partials in block order (a fixed order).
+// Expert-in (A).  A unit is one union expert e and one 128-row tile of W_in_e
+// (d_e = 128: the whole expert).  The pair at position p of the A order takes
+// units p, p + #pairs, ...; its block of rank r in the pair multiplies the
+// k-half r of W_in_e (tcgen05; weights as the M = 128 operand, the chunk's N
+// tokens as N) into a TMEM accumulator.  The two blocks split the tokens: each
+// sends the peer its partial for the peer's half with st.async straight into
+// the peer's shared memory (the bytes are counted on the peer's mbarrier), adds
+// the peer's partial for its own half, applies the post-hoc mask, the gate and
+// Swish, writes its half of h' (bf16) to global memory and counts it in for the
+// expert.  The A order lists first the pairs whose cluster has no expert-out
+// row tile, so that those clusters start expert-out work with free hands.
+//
+// Expert-out (B).  y^T = sum_e W_out_e h'_e^T with W_out_e's 128-row tiles as the
+// M operand and the tokens as N.  Cluster c owns the row tiles c, c + #clusters,
+// ...; each of its 4 blocks takes a quarter of a row tile's (expert, 64-wide
+// k-block) tiles.  A tile waits (bounded) until every expert's h' is counted
+// in, then its h' slice arrives by TMA.  The 4 partial tiles are summed inside
+// the cluster: warp q of every block st.async's its 32 accumulator rows to the
+// block of rank q, which adds the 4 contributions in rank order (a fixed order)
+// and writes those 32 rows of y.
 //
 // Roles (224 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM owner
-// and h' loader, warps 3-6 epilogue (warp 4 also finishes the A units).  Every
-// wait is bounded; a timeout records BLOCKFFN_ERR_TIMEOUT and the block winds
-// down without leaving copies in flight.
+// and h' loader, warps 3-6 epilogue.  Every wait is bounded; a timeout records
+// BLOCKFFN_ERR_TIMEOUT and the block winds down without leaving copies in
+// flight.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -45,14 +48,18 @@
 namespace bffn {
 
 constexpr int kRsThreads = 224;
+constexpr int kRsCluster = 4;
 constexpr int kRsStages = 10;
 constexpr int kRsStageBytes = 16384 + 4096;  // weight tile [128 x 64] + activation tile [<=32 x 64]
-constexpr int kRsNAccB = 4;                  // expert-out accumulators (32 columns each)
-constexpr int kRsTmemCols = 256;             // 2 x 32 expert-in + 4 x 32 expert-out columns
+constexpr int kRsTmemCols = 128;             // 2 expert-in + 2 expert-out accumulators of <=32 columns
 constexpr int kRsMaxE = 256;
 constexpr int kRsMaxG = 160;
-constexpr int kRsPartBytes = 16 * 128 * 4;   // fp32 partial h^T for the peer's half [<=16 tokens][128 rows]
-constexpr int kRsHStageBytes = 16 * 128 * 2; // this block's half of h' [<=16 tokens][128 rows] bf16
+// receive area: two expert-in partials for this block's half of the tokens
+// ([<=16 tokens][128 rows] fp32 each); later the expert-out quadrant partials
+// from the other 3 ranks ([4 slots][32 rows][<=32 tokens] fp32) reuse it
+constexpr int kRsRecvBytes = 2 * 16 * 128 * 4;
+constexpr int kRsHStageBytes = 16 * 128 * 2;  // this block's half of h' [<=16 tokens][128 rows] bf16
+static_assert(4 * 32 * 32 * 4 <= kRsRecvBytes, "expert-out quadrants fit the receive area");
 
 struct RsShared {
     uint64_t full_w[kRsStages];   // TMA bytes landed
@@ -60,32 +67,32 @@ struct RsShared {
     uint64_t empty[kRsStages];    // MMAs reading the stage are done
     uint64_t accA_full[2];
     uint64_t accA_empty[2];
-    uint64_t accB_full[kRsNAccB];
-    uint64_t accB_empty[kRsNAccB];
-    uint64_t part_ready;          // 2 arrivals: both blocks of the pair wrote their partial
-    uint64_t part_free;           // 1 arrival: the peer finished reading this block's partial
+    uint64_t accB_full[2];
+    uint64_t accB_empty[2];
+    uint64_t recvA[2];            // the peer's expert-in partial landed here (st.async bytes)
+    uint64_t freeA[2];            // 1 arrival: the peer has read what this block sent it
+    uint64_t recvB;               // the other ranks' expert-out quadrant partials landed
+    uint64_t freeB;               // 3 arrivals: the other ranks have summed the last quadrants sent them
     uint64_t mma_done;
     uint64_t a_pub;               // 1 arrival: this block's expert-in results are published
     uint32_t tmem_base;
     volatile int abort;
     uint32_t epoch;
     int P;
-    int ep_wait[2];
     int ep_ok;
     uint32_t trace_once;          // trace slots already stamped (first occurrence only)
+    int pendA[2], pendB;          // parity of a receive phase armed but not seen complete, or -1
     float s_gate[2][32];          // gates of the current expert-in unit's expert, per token
-    int s_contrib[kRsMaxG];
-    long long s_blo[kRsMaxG + 1];   // first expert-out tile of every block
-    int32_t s_pair_e[kRsMaxE];
-    uint32_t s_tmask[kRsMaxE];
+    int32_t s_pair_e[kRsMaxE];    // the union, ascending
+    uint32_t s_tmask[kRsMaxE];    // per expert: bit t = token t's gate is nonzero
     uint32_t s_bal[kRsMaxE / 32];
 };
 
 enum : int {
     kRtStart = 0, kRtPrologue = 1, kRtFirstLoad = 2, kRtLastLoad = 3, kRtFirstFull = 4,
     kRtLastACommit = 5, kRtADone = 7, kRtFirstFlag = 8, kRtLastFlag = 9, kRtLastCommit = 10,
-    kRtLastEpi = 11, kRtEnd = 13, kRtATmem = 14, kRtAPart = 15, kRtAReady = 16, kRtARead = 17,
-    kRtAWritten = 18, kRtBPartial = 21, kRtBReduced = 23, kRtFirstBMma = 24, kRtSlots = 64
+    kRtLastEpi = 11, kRtEnd = 13, kRtATmem = 14, kRtASent = 15, kRtAReady = 16, kRtARead = 17,
+    kRtAWritten = 18, kRtBSent = 21, kRtBReduced = 23, kRtFirstBMma = 24, kRtSlots = 64
 };
 #define RS_TRACE(slot) \
     do { if (a.trace) a.trace[(size_t)blockIdx.x * kRtSlots + (slot)] = globaltimer_ns(); } while (0)
@@ -96,17 +103,6 @@ enum : int {
     } while (0)
 
 __device__ __forceinline__ float rs_swish(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
-
-// block holding expert-out tile j: the last i with blo[i] <= j (ranges may be empty)
-__device__ __forceinline__ int rs_owner(const long long* blo, int G, long long j) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (blo[mid] <= j) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
 
 // Position in the ring of pipeline stages: the stage and the parity of its
 // current use, stepped without divisions.
@@ -121,47 +117,83 @@ struct RingPos {
     }
 };
 
-// Expert-out tile j = (rt * P + s) * KBe + kb (row tile, expert slot, k-block),
-// stepped without divisions.
-struct BTile {
-    int rt, s, kb;
-    __device__ __forceinline__ void init(long long j, int P, int KBe) {
-        const long long per = (long long)P * KBe;
-        rt = (int)(j / per);
-        const int rem = (int)(j - (long long)rt * per);
-        s = rem / KBe;
-        kb = rem - s * KBe;
+// This block's expert-out tiles, in order: for each row tile rt = cid, cid +
+// #clusters, ... (< RT), the tiles j in [lo, hi) of that row tile, tile j being
+// expert slot j / KBe and 64-wide k-block j % KBe.  Stepped without divisions.
+struct BCursor {
+    int rt, j, s, kb;
+    int lo, hi, s0, kb0, step, KBe;
+    __device__ __forceinline__ void init(int cid, int ncl, int lo_, int hi_, int KBe_) {
+        rt = cid;
+        step = ncl;
+        lo = lo_;
+        hi = hi_;
+        KBe = KBe_;
+        s0 = lo / KBe;
+        kb0 = lo - s0 * KBe;
+        j = lo;
+        s = s0;
+        kb = kb0;
     }
-    __device__ __forceinline__ void advance(int P, int KBe) {
-        if (++kb == KBe) {
+    __device__ __forceinline__ void advance() {
+        if (++j == hi) {
+            j = lo;
+            s = s0;
+            kb = kb0;
+            rt += step;
+        } else if (++kb == KBe) {
             kb = 0;
-            if (++s == P) {
-                s = 0;
-                ++rt;
-            }
+            ++s;
         }
     }
 };
+
+// Where this block stands in the grid and what it computes.
+struct RsWork {
+    int cr, cid, ncl, pr, hk;   // cluster rank, cluster, #clusters, pair, k-half
+    int nA, apos, npairs;       // expert-in units of the pair: v = apos + u * npairs, u < nA
+    int nRT;                    // expert-out row tiles owned by the cluster
+    int bLo, bHi;               // this block's tiles of each of them
+};
+
+__device__ __forceinline__ RsWork rs_work(int G, int P, int MT, int KBe, int RT) {
+    RsWork w;
+    w.cr = (int)cluster_ctarank();
+    w.cid = (int)blockIdx.x / kRsCluster;
+    w.ncl = G / kRsCluster;
+    w.pr = w.cid * 2 + (w.cr >> 1);
+    w.hk = w.cr & 1;
+    w.npairs = 2 * w.ncl;
+    // the A order: pairs of clusters without a row tile first
+    const int nBc = min(RT, w.ncl);
+    w.apos = w.pr >= 2 * nBc ? w.pr - 2 * nBc : w.pr + 2 * (w.ncl - nBc);
+    const int VA = P * MT;
+    w.nA = w.apos < VA ? (VA - w.apos + w.npairs - 1) / w.npairs : 0;
+    w.nRT = w.cid < RT ? (RT - w.cid + w.ncl - 1) / w.ncl : 0;
+    const int per_rt = P * KBe;
+    w.bLo = per_rt * w.cr / kRsCluster;
+    w.bHi = per_rt * (w.cr + 1) / kRsCluster;
+    return w;
+}
 
 template <int N>
 __global__ void __launch_bounds__(kRsThreads, 1)
 union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_win,
                     const __grid_constant__ CUtensorMap tm_wout, const __grid_constant__ CUtensorMap tm_h,
-                    const DcArgs a) {
+                    const __grid_constant__ CUtensorMap tm_y, const DcArgs a) {
+    constexpr int NH = N / 2;   // tokens per k-half block in the expert-in epilogue
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float* part = reinterpret_cast<float*>(smem + kRsStages * kRsStageBytes);     // [N][128] fp32
-    __nv_bfloat16* hstage = reinterpret_cast<__nv_bfloat16*>(smem + kRsStages * kRsStageBytes + kRsPartBytes);
-    RsShared& sh = *reinterpret_cast<RsShared*>(smem + kRsStages * kRsStageBytes + kRsPartBytes + kRsHStageBytes);
+    float* recv = reinterpret_cast<float*>(smem + kRsStages * kRsStageBytes);
+    __nv_bfloat16* hstage = reinterpret_cast<__nv_bfloat16*>(smem + kRsStages * kRsStageBytes + kRsRecvBytes);
+    RsShared& sh = *reinterpret_cast<RsShared*>(smem + kRsStages * kRsStageBytes + kRsRecvBytes + kRsHStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = gridDim.x, cta = blockIdx.x;
+    const int G = gridDim.x;
     const int KBe = a.d_e / 64;     // 64-wide k-blocks of one expert in the expert-out GEMM
     const int MT = a.d_e / 128;     // 128-row tiles of W_in_e
     const int KBh = a.KB / 2;       // k-tiles of one k-half
-    const int NCL = G / 2;          // pairs
-    const int pr = cta >> 1;        // this block's pair
-    const int hk = cta & 1;         // its rank in the pair = its k-half
+    const int nt = min(a.n, a.T);
 
     if (threadIdx.x == 0) {
         RS_TRACE(kRtStart);
@@ -173,25 +205,35 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sh.accA_full[s], 1);
             mbar_init(&sh.accA_empty[s], 1);
-        }
-        for (int s = 0; s < kRsNAccB; ++s) {
             mbar_init(&sh.accB_full[s], 1);
             mbar_init(&sh.accB_empty[s], 4);
+            mbar_init(&sh.recvA[s], 1);
+            mbar_init(&sh.freeA[s], 1);
         }
-        mbar_init(&sh.part_ready, 2);
-        mbar_init(&sh.part_free, 1);
+        mbar_init(&sh.recvB, 1);
+        mbar_init(&sh.freeB, 3);
         mbar_init(&sh.mma_done, 1);
         mbar_init(&sh.a_pub, 1);
         sh.trace_once = 0u;
+        sh.pendA[0] = sh.pendA[1] = sh.pendB = -1;
         fence_mbar_init();
         const int32_t st0 = __ldcg(&a.ctl->status);
-        const uint32_t ep0 = __ldcg(&a.ctl->epoch);
+        // acquire: the read is done before this block's count below is seen
+        const uint32_t ep0 = ld_acquire_gpu(&a.ctl->epoch);
         sh.abort = st0 != 0;
         sh.epoch = ep0;
+        // The last block to read the launch counter advances it for the next
+        // launch (every block of this one has read it by then; the next launch
+        // sees the new value because it starts after this one ends).
+        if (atomicAdd(&a.ctl->done, 1u) == (uint32_t)(gridDim.x - 1)) {
+            a.ctl->done = 0u;
+            a.ctl->epoch = ep0 + 1u;
+        }
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_win);
         prefetch_tmap(&tm_wout);
         prefetch_tmap(&tm_h);
+        prefetch_tmap(&tm_y);
     }
     if (warp == 2) {
         tmem_alloc(&sh.tmem_base, kRsTmemCols);
@@ -200,7 +242,6 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     if (warp >= 3) {
         // the chunk's union, ascending (warps 3-6 take 32-expert groups; all of a
         // lane's gate loads are issued before their first use)
-        const int nt = min(a.n, a.T);
         const int ngroups = (a.E + 31) / 32;
         for (int g = warp - 3; g < ngroups; g += 4) {
             const int e = g * 32 + lane;
@@ -224,39 +265,30 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 base += __popc(bal);
             }
             if (lane == 0) sh.P = base;
-            // Expert-out tile ranges: an even split over all blocks.  The expert-out
-            // MMAs all run after the h' hand-off, so it is their count per block
-            // that sets the length of that phase; the expert-in blocks load their
-            // share after publishing h' (their weights were sent towards L2 early).
-            const long long NB = (long long)a.RT * base * KBe;
-            for (int i = lane; i < G; i += 32) sh.s_blo[i] = NB * i / G;
-            if (lane == 0) sh.s_blo[G] = NB;
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    cluster_barrier_sync();   // the peer's barriers are initialised before any remote arrival
+    const int P = sh.P;
+    const RsWork wk = rs_work(G, P, MT, KBe, a.RT);
+    const int nBt = wk.bHi - wk.bLo;                 // expert-out tiles per owned row tile
+    const int totB = P > 0 ? wk.nRT * nBt : 0;        // this block's expert-out tiles
+    const bool doB = P > 0 && wk.nRT > 0;             // this cluster sums expert-out row tiles
+    if (threadIdx.x == 0 && doB) {
+        // the first expert-out reduction: 3 quadrant partials of 32 rows x N tokens
+        mbar_arrive_expect_tx(&sh.recvB, 3u * 32u * N * 4u);
+        sh.pendB = 0;
+    }
+    cluster_barrier_sync();   // every block's barriers are initialised before any remote arrival
     if (threadIdx.x == 0) RS_TRACE(kRtPrologue);
 
     const uint32_t tmem = sh.tmem_base;
-    const int P = sh.P;
     const int par = (int)(sh.epoch & 1u);
     uint32_t* const readyA = a.readyA + (size_t)par * a.E;
-    const int VA = P * MT;                                          // A units (expert, 128-row tile)
-    const int nA = VA / NCL + (pr < VA % NCL ? 1 : 0);               // A units of this pair
-    const long long bLo = sh.s_blo[cta], bHi = sh.s_blo[cta + 1];
-    const long long per_rt = (long long)P * KBe;                     // expert-out tiles per row tile
     const uint64_t limit_peer = a.wait_ns;
     const uint64_t limit = 2 * a.wait_ns;
-    const uint32_t accA_col = 0, accB_col = 64;
-
-    // expert-out segments: a row tile rt is the unit, tiles [rt*per_rt, (rt+1)*per_rt)
-    auto seg_of = [&](long long j, long long& first, long long& last, int& rt) {
-        rt = (int)(j / per_rt);
-        first = (long long)rt * per_rt;
-        last = first + per_rt - 1;
-    };
+    const uint32_t accA_col = 0, accB_col = 2 * N;
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer --
@@ -266,11 +298,11 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             long long i = 0;
             RingPos rp;
             bool stop = false;
-            for (int ua = 0; ua < nA && !stop; ++ua) {
-                const int v = pr + ua * NCL;
+            for (int ua = 0; ua < wk.nA && !stop; ++ua) {
+                const int v = wk.apos + ua * wk.npairs;
                 const int e = sh.s_pair_e[v / MT], mt = v % MT;
                 for (int t = 0; t < KBh; ++t, ++i, rp.advance()) {
-                    const int kt = hk * KBh + t;
+                    const int kt = wk.hk * KBh + t;
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
                         stop = true;
                         break;
@@ -283,34 +315,27 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 }
             }
             // Expert-out weights.  A block with expert-in units sends all of its
-            // tiles towards L2 now and loads them into the ring only after its h' is
-            // published: a release waits for the block's bulk loads in flight, and
-            // no expert-out MMA can start before every h' is out anyway.  Other
-            // blocks load at once and prefetch what the ring cannot hold yet.
-            {
-                const long long nB = bHi - bLo;
-                const long long j0 = nA > 0 ? bLo : bHi - min(nB, max(0LL, nB - (long long)kRsStages));
-                if (j0 < bHi) {
-                    BTile bt;
-                    bt.init(j0, P, KBe);
-                    for (long long j = j0; j < bHi; ++j, bt.advance(P, KBe))
-                        tma_prefetch_l2_2d(&tm_wout, bt.kb * 64, sh.s_pair_e[bt.s] * a.d_h + bt.rt * 128);
-                }
-                if (nA > 0 && bLo < bHi && !stop &&
-                    !wait_bar(&sh.a_pub, 0u, limit, &sh.abort, a.ctl, kWaitEmpty))
+            // tiles towards L2 now and loads them into the ring only after its h'
+            // is published: a release waits for the block's bulk loads in flight,
+            // and no expert-out MMA can start before every h' is out anyway.
+            // Other blocks load at once and prefetch what the ring cannot hold yet.
+            if (totB > 0) {
+                BCursor bc;
+                bc.init(wk.cid, wk.ncl, wk.bLo, wk.bHi, KBe);
+                for (int q = 0; q < totB; ++q, bc.advance())
+                    if (wk.nA > 0 || q >= kRsStages)
+                        tma_prefetch_l2_2d(&tm_wout, bc.kb * 64, sh.s_pair_e[bc.s] * a.d_h + bc.rt * 128);
+                if (wk.nA > 0 && !stop && !wait_bar(&sh.a_pub, 0u, limit, &sh.abort, a.ctl, kWaitEmpty))
                     stop = true;
-            }
-            if (bLo < bHi) {
-                BTile bt;
-                bt.init(bLo, P, KBe);
-                for (long long j = bLo; j < bHi && !stop; ++j, ++i, rp.advance(), bt.advance(P, KBe)) {
+                bc.init(wk.cid, wk.ncl, wk.bLo, wk.bHi, KBe);
+                for (int q = 0; q < totB && !stop; ++q, ++i, rp.advance(), bc.advance()) {
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
                         stop = true;
                         break;
                     }
                     mbar_arrive_expect_tx(&sh.full_w[rp.st], 16384);
-                    tma_load_2d(smem + rp.st * kRsStageBytes, &tm_wout, &sh.full_w[rp.st], bt.kb * 64,
-                                sh.s_pair_e[bt.s] * a.d_h + bt.rt * 128, pol_stream);
+                    tma_load_2d(smem + rp.st * kRsStageBytes, &tm_wout, &sh.full_w[rp.st], bc.kb * 64,
+                                sh.s_pair_e[bc.s] * a.d_h + bc.rt * 128, pol_stream);
                     if (i == 0) RS_TRACE(kRtFirstLoad);
                 }
             }
@@ -325,13 +350,13 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             long long i = 0;
             RingPos rp;
             bool stop = sh.abort != 0;
-            for (int ua = 0; ua < nA && !stop; ++ua) {
+            for (int ua = 0; ua < wk.nA && !stop; ++ua) {
                 const int ab = ua & 1;
                 if (!wait_bar(&sh.accA_empty[ab], (uint32_t)(((ua >> 1) & 1) ^ 1), limit, &sh.abort, a.ctl,
                               kWaitAccEmpty))
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem + accA_col + (uint32_t)(ab * 32);
+                const uint32_t d = tmem + accA_col + (uint32_t)(ab * N);
                 for (int t = 0; t < KBh; ++t, ++i, rp.advance()) {
                     const int st = rp.st;
                     if (!wait_bar(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
@@ -353,20 +378,15 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 umma_commit(&sh.accA_full[ab]);
                 RS_TRACE(kRtLastACommit);
             }
-            uint32_t acc_i = 0;
-            long long j = bLo;
-            while (!stop && j < bHi) {
-                long long first, last;
-                int rt;
-                seg_of(j, first, last, rt);
-                const long long shi = min(bHi, last + 1);
-                const int ab = (int)(acc_i % kRsNAccB);
-                if (!wait_bar(&sh.accB_empty[ab], ((acc_i / kRsNAccB) & 1u) ^ 1u, limit, &sh.abort, a.ctl,
+            // one accumulator per owned row tile, alternating between two
+            for (int k = 0; k < (totB > 0 ? wk.nRT : 0) && !stop; ++k) {
+                const int ab = k & 1;
+                if (!wait_bar(&sh.accB_empty[ab], (uint32_t)(((k >> 1) & 1) ^ 1), limit, &sh.abort, a.ctl,
                               kWaitAccEmpty))
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem + accB_col + (uint32_t)(ab * 32);
-                for (long long jj = j; jj < shi; ++jj, ++i, rp.advance()) {
+                const uint32_t d = tmem + accB_col + (uint32_t)(ab * N);
+                for (int q = 0; q < nBt; ++q, ++i, rp.advance()) {
                     const int st = rp.st;
                     if (!wait_bar(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
                         !wait_bar(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
@@ -374,20 +394,18 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         break;
                     }
                     tc_fence_after();
-                    if (jj == bLo) RS_TRACE(kRtFirstBMma);
+                    if (k == 0 && q == 0) RS_TRACE(kRtFirstBMma);
                     const uint32_t wb = smem_u32(smem + st * kRsStageBytes);
                     const uint32_t hb = wb + 16384;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_bf16(d, sw128_kmajor_desc(wb + kk * 32), sw128_kmajor_desc(hb + kk * 32), idesc,
-                                  (jj > j || kk > 0) ? 1u : 0u);
+                                  (q > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sh.empty[st]);
                 }
                 if (stop) break;
                 umma_commit(&sh.accB_full[ab]);
                 RS_TRACE(kRtLastCommit);
-                ++acc_i;
-                j = shi;
             }
             umma_commit(&sh.mma_done);
         }
@@ -397,8 +415,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // tile the warp waits (bounded) until every expert slot's h' is counted in;
         // then lane 0 moves each tile's [N x 64] h' slice with one TMA load, which
         // lands in the same 128-byte-swizzled layout as the weight tile's operand.
-        const long long nAt = (long long)nA * KBh;
-        const long long total_tiles = nAt + (bHi - bLo);
+        const long long nAt = (long long)wk.nA * KBh;
         long long i = 0;
         RingPos rp;
         int stop = sh.abort != 0;
@@ -412,7 +429,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
         }
         stop = __shfl_sync(0xffffffffu, stop, 0);
-        if (!stop && total_tiles > nAt) {
+        if (!stop && totB > 0) {
             // The expert-in units all finish at about the same time, so one combined
             // wait costs no more than the slowest slot; each poll round checks 32
             // slots at once (one acquire load per lane).
@@ -442,13 +459,13 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 RS_TRACE_ONCE(kRtFirstFlag);
                 RS_TRACE(kRtLastFlag);
                 const uint64_t pol = policy_evict_first();
-                BTile bt;
-                bt.init(bLo, P, KBe);
-                for (; i < total_tiles; ++i, rp.advance(), bt.advance(P, KBe)) {
+                BCursor bc;
+                bc.init(wk.cid, wk.ncl, wk.bLo, wk.bHi, KBe);
+                for (int q = 0; q < totB; ++q, ++i, rp.advance(), bc.advance()) {
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) break;
                     mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 128));
-                    tma_load_2d(smem + rp.st * kRsStageBytes + 16384, &tm_h, &sh.full_h[rp.st], bt.kb * 64,
-                                bt.s * N, pol);
+                    tma_load_2d(smem + rp.st * kRsStageBytes + 16384, &tm_h, &sh.full_h[rp.st], bc.kb * 64,
+                                bc.s * N, pol);
                 }
                 // no copy into this block's shared memory outlives it
                 for (long long q = i - kRsStages < nAt ? nAt : i - kRsStages; q < i; ++q)
@@ -457,308 +474,272 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         }
     } else {
         // --------------------------------------------------------- epilogue --
-        const int qd = warp & 3;
+        const int qd = warp & 3;                     // TMEM lane quadrant of this warp
         const int row = qd * 32 + lane;              // TMEM lane = accumulator row
         const int et = threadIdx.x - 96;             // 0..127
         {
             // zero the other parity's counters for the next launch
             const int oth = par ^ 1;
-            for (int k2 = cta * 128 + et; k2 < a.E; k2 += G * 128) a.readyA[(size_t)oth * a.E + k2] = 0u;
+            for (int k2 = (int)blockIdx.x * 128 + et; k2 < a.E; k2 += G * 128) a.readyA[(size_t)oth * a.E + k2] = 0u;
         }
         bool failed = sh.abort != 0;
-        const int nt = min(a.n, a.T);
-        if (P == 0 && cta == 0 && !failed) {
+        if (P == 0 && blockIdx.x == 0 && !failed) {
             // empty union: y is all zeros
             for (size_t k2 = et; k2 < (size_t)nt * a.d_h; k2 += 128) a.y[k2] = __float2bfloat16_rn(0.f);
         }
-        // ---- A units: the pair's two k-half partials meet in shared memory
-        {
-            const uint32_t peer = (uint32_t)(hk ^ 1);
-            const uint32_t peer_part = mapa_shared(smem_u32(part), peer);
-            const uint32_t peer_ready = mapa_shared(smem_u32(&sh.part_ready), peer);
-            const uint32_t own_ready = mapa_shared(smem_u32(&sh.part_ready), (uint32_t)hk);
-            const uint32_t peer_free = mapa_shared(smem_u32(&sh.part_free), peer);
-            for (int ua = 0; ua < nA && !failed; ++ua) {
-                const int ab = ua & 1;
-                const int v = pr + ua * NCL;
-                const int s = v / MT, mt = v % MT;
-                const int e = sh.s_pair_e[s];
-                // stage the unit's gates now: the accumulator wait hides their latency,
-                // and the activation loop below then reads shared memory only
-                if (et < 32) sh.s_gate[ab][et] = a.gates[(size_t)min(et, nt - 1) * a.E + e];
-                if (et == 0) {
-                    int ok = wait_bar(&sh.accA_full[ab], (uint32_t)((ua >> 1) & 1), limit, &sh.abort, a.ctl,
-                                      kWaitAccFull) ? 1 : 0;
-                    // the peer finished reading this block's previous partial
-                    if (ok && ua > 0)
-                        ok = wait_bar_cluster(&sh.part_free, (uint32_t)((ua - 1) & 1), limit_peer, &sh.abort,
-                                              a.ctl, kWaitPeers) ? 1 : 0;
-                    sh.ep_ok = ok;
-                }
-                named_bar_sync(1, 128);
-                if (!sh.ep_ok) { failed = true; break; }
-                tc_fence_after();
-                uint32_t r[32];
-                const uint32_t taddr = tmem + ((uint32_t)(qd * 32) << 16) + accA_col + (uint32_t)(ab * 32);
-                if constexpr (N == 32) tmem_ld_32x32b_x32(taddr, r);
-                else tmem_ld_32x32b_x16(taddr, r);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.accA_empty[ab]);
-                if (et == 0) RS_TRACE_ONCE(kRtATmem);
-                // The pair splits the chunk's tokens: this block finishes tokens
-                // [tg, tg + NH) of all 128 rows and the peer the other half.  Each block
-                // hands the peer its partial for the peer's tokens: float4 of the half's
-                // tokens 4k..4k+3 of a row at k*128 + row.
-                constexpr int NH = N / 2;
-                const int tg = hk * NH;
-                {
-                    float4* p4 = reinterpret_cast<float4*>(part) + row;
-#pragma unroll
-                    for (int k4 = 0; k4 < NH / 4; ++k4) {
-                        float f[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            f[u] = __uint_as_float(hk ? r[4 * k4 + u] : r[NH + 4 * k4 + u]);
-                        p4[k4 * 128] = make_float4(f[0], f[1], f[2], f[3]);
-                    }
-                }
-                const uint32_t bits = sh.s_tmask[e] >> tg;   // this half's token bits
-                named_bar_sync(1, 128);
-                if (et == 0) {
-                    RS_TRACE_ONCE(kRtAPart);
-                    mbar_arrive_cluster(own_ready);
-                    mbar_arrive_cluster(peer_ready);
-                    sh.ep_ok = wait_bar_cluster(&sh.part_ready, (uint32_t)(ua & 1), limit_peer, &sh.abort, a.ctl,
-                                                kWaitPeers) ? 1 : 0;
-                    RS_TRACE_ONCE(kRtAReady);
-                }
-                named_bar_sync(1, 128);
-                if (!sh.ep_ok) { failed = true; break; }
-                // h = (k-half 0) + (k-half 1): two terms, and the sum does not depend on
-                // which block of the pair forms it
-                float z[NH];
-                {
-                    float4 pv[NH / 4];
-#pragma unroll
-                    for (int k4 = 0; k4 < NH / 4; ++k4)
-                        pv[k4] = ld_shared_cluster_f4(peer_part + (uint32_t)((k4 * 128 + row) * 16));
-#pragma unroll
-                    for (int k4 = 0; k4 < NH / 4; ++k4) {
-                        const float pw[4] = {pv[k4].x, pv[k4].y, pv[k4].z, pv[k4].w};
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            z[4 * k4 + u] = __uint_as_float(hk ? r[NH + 4 * k4 + u] : r[4 * k4 + u]) + pw[u];
-                    }
-                }
-                named_bar_sync(1, 128);
-                if (et == 0) {
-                    RS_TRACE_ONCE(kRtARead);
-                    mbar_arrive_cluster(peer_free);   // done with the peer's partial
-                }
-                // h' = bit ? g * Swish(h) : 0 (a select, so a masked token gives 0 even if
-                // its h is not finite), staged token-major in shared memory, then written
-                // with 16-byte stores: token t's 128 rows are 256 contiguous bytes
-                {
-                    __nv_bfloat16* stg = hstage + row;
-#pragma unroll
-                    for (int tl = 0; tl < NH; ++tl) {
-                        const float gsw = sh.s_gate[ab][tg + tl] * rs_swish(z[tl]);
-                        stg[tl * 128] = __float2bfloat16_rn(((bits >> tl) & 1u) ? gsw : 0.f);
-                    }
-                }
-                named_bar_sync(1, 128);
-                {
-                    const uint4* src4 = reinterpret_cast<const uint4*>(hstage);
-                    for (int c = et; c < NH * 16; c += 128) {
-                        const int tl = c >> 4, c16 = c & 15;
-                        uint4* dst4 =
-                            reinterpret_cast<uint4*>(a.hbuf + ((size_t)s * N + tg + tl) * a.d_e + mt * 128) + c16;
-                        *dst4 = src4[c];
-                    }
-                }
-                // one release for the whole block: the barrier orders every thread's
-                // stores before thread 0's releasing count
-                named_bar_sync(1, 128);
-                if (et == 0) {
-                    if ((v * 2 + hk) != a.skip_unit) red_release_add_gpu(&readyA[s], 1u);
-                    RS_TRACE_ONCE(kRtAWritten);
-                }
-            }
+        // ---- A units: each block finishes its half of the tokens
+        const uint32_t peer = (uint32_t)(wk.cr ^ 1);
+        const uint32_t peer_recv = mapa_shared(smem_u32(recv), peer);
+        const uint32_t peer_recvA = mapa_shared(smem_u32(&sh.recvA[0]), peer);
+        const uint32_t peer_freeA = mapa_shared(smem_u32(&sh.freeA[0]), peer);
+        const int tg = wk.hk * NH;                   // first token this block finishes
+        for (int ua = 0; ua < wk.nA && !failed; ++ua) {
+            const int b = ua & 1;
+            const int v = wk.apos + ua * wk.npairs;
+            const int s = v / MT, mt = v % MT;
+            const int e = sh.s_pair_e[s];
+            // stage the unit's gates now: the accumulator wait hides their latency,
+            // and the activation loop below then reads shared memory only
+            if (et < 32) sh.s_gate[b][et] = a.gates[(size_t)min(et, nt - 1) * a.E + e];
             if (et == 0) {
-                RS_TRACE(kRtADone);
-                if (nA > 0) mbar_arrive(&sh.a_pub);   // the producer may load expert-out tiles now
+                // the peer's partial for this block's half of unit ua lands in buffer b
+                mbar_arrive_expect_tx(&sh.recvA[b], (uint32_t)(NH * 128 * 4));
+                sh.pendA[b] = (ua >> 1) & 1;
+                int ok = wait_bar(&sh.accA_full[b], (uint32_t)((ua >> 1) & 1), limit, &sh.abort, a.ctl,
+                                  kWaitAccFull) ? 1 : 0;
+                // before sending into the peer's buffer b again, the peer has read it
+                if (ok && ua >= 2)
+                    ok = wait_bar_cluster(&sh.freeA[b], (uint32_t)(((ua - 2) >> 1) & 1), limit_peer, &sh.abort,
+                                          a.ctl, kWaitPeers) ? 1 : 0;
+                sh.ep_ok = ok;
             }
-        }
-        // ---- expert-out row tiles.  A row tile whose k-range is split over several
-        // blocks is summed without a flag: every contributor stores its partial as
-        // (launch tag, fp32) pairs with relaxed stores, and the block that sums a
-        // slice of the tile's rows polls those pairs until each carries this
-        // launch's tag, then adds the contributors in block order.
-        const uint32_t tag = sh.epoch + 1u;
-        const unsigned long long tag_hi = (unsigned long long)tag << 32;
-        const size_t slot_pairs = (size_t)(N / 2) * 128;   // 16-byte pairs in one partial slot
-        ulonglong2* const partD = reinterpret_cast<ulonglong2*>(a.partD);
-        auto contributors = [&](long long first, long long last, int& q0, int& q1, int& n, int& rank) {
-            q0 = rs_owner(sh.s_blo, G, first);
-            q1 = rs_owner(sh.s_blo, G, last);
-            n = 0;
-            rank = -1;
-            for (int qq = q0; qq <= q1; ++qq) {
-                if (sh.s_blo[qq + 1] > sh.s_blo[qq]) {
-                    if (qq == cta) rank = n;
-                    ++n;
-                }
-            }
-        };
-        long long pend_first[2], pend_last[2];
-        int pend_rt[2];
-        int npend = 0;
-        uint32_t acc_i = 0;
-        long long j = bLo;
-        failed = failed || sh.abort;
-        while (!failed && j < bHi) {
-            long long first, last;
-            int rt;
-            seg_of(j, first, last, rt);
-            const long long shi = min(bHi, last + 1);
-            const int ab = (int)(acc_i % kRsNAccB);
-            if (et == 0)
-                sh.ep_wait[acc_i & 1u] =
-                    wait_bar(&sh.accB_full[ab], (acc_i / kRsNAccB) & 1u, limit, &sh.abort, a.ctl, kWaitAccFull)
-                        ? 1 : 0;
             named_bar_sync(1, 128);
-            if (!sh.ep_wait[acc_i & 1u]) { failed = true; break; }
+            if (!sh.ep_ok) { failed = true; break; }
             tc_fence_after();
             uint32_t r[32];
-            const uint32_t taddr = tmem + ((uint32_t)(qd * 32) << 16) + accB_col + (uint32_t)(ab * 32);
+            const uint32_t taddr = tmem + ((uint32_t)(qd * 32) << 16) + accA_col + (uint32_t)(b * N);
             if constexpr (N == 32) tmem_ld_32x32b_x32(taddr, r);
             else tmem_ld_32x32b_x16(taddr, r);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.accB_empty[ab]);
-            ++acc_i;
-            int q0, q1, nc, rank;
-            contributors(first, last, q0, q1, nc, rank);
-            if (nc == 1) {
-                __nv_bfloat16* ycol = a.y + rt * 128 + row;
+            if (lane == 0) mbar_arrive(&sh.accA_empty[b]);
+            if (et == 0) RS_TRACE_ONCE(kRtATmem);
+            // the peer's half of the tokens goes to the peer: float4 of the half's
+            // tokens 4k..4k+3 of a row at k*128 + row of its buffer b
+            {
+                const uint32_t dst = peer_recv + (uint32_t)(b * NH * 128 * 4 + row * 16);
+                const uint32_t rbar = peer_recvA + (uint32_t)(b * 8);
 #pragma unroll
-                for (int t = 0; t < N; ++t)
-                    if (t < nt) ycol[(size_t)t * a.d_h] = __float2bfloat16_rn(__uint_as_float(r[t]));
-                if (et == 0) RS_TRACE(kRtLastEpi);
-            } else {
-                // pair kp of a row holds tokens 2kp and 2kp+1: [kp][row] x 16 bytes
-                const int myslot = bLo >= first ? 0 : 1;
-                ulonglong2* dst = partD + (size_t)(cta * 2 + myslot) * slot_pairs + row;
+                for (int k4 = 0; k4 < NH / 4; ++k4) {
+                    float f[4];
 #pragma unroll
-                for (int kp = 0; kp < N / 2; ++kp)
-                    st_relaxed_v2_b64(dst + kp * 128, tag_hi | r[2 * kp], tag_hi | r[2 * kp + 1]);
-                if (et == 0) RS_TRACE_ONCE(kRtBPartial);
-                if (npend < 2) {
-                    pend_first[npend] = first;
-                    pend_last[npend] = last;
-                    pend_rt[npend] = rt;
-                    ++npend;
+                    for (int u = 0; u < 4; ++u)
+                        f[u] = __uint_as_float(wk.hk ? r[4 * k4 + u] : r[NH + 4 * k4 + u]);
+                    st_async_v4(dst + (uint32_t)(k4 * 128 * 16), f[0], f[1], f[2], f[3], rbar);
                 }
             }
-            j = shi;
-        }
-        // second pass: sum my slice of each split row tile's rows
-        for (int pi = 0; pi < npend && !failed; ++pi) {
-            int q0, q1, nc, rank;
-            contributors(pend_first[pi], pend_last[pi], q0, q1, nc, rank);
-            const int rt = pend_rt[pi];
+            if (et == 0) RS_TRACE_ONCE(kRtASent);
+            const uint32_t bits = sh.s_tmask[e] >> tg;   // this half's token bits
             if (et == 0) {
-                int k2 = 0;
-                for (int qq = q0; qq <= q1 && k2 < kRsMaxG; ++qq)
-                    if (sh.s_blo[qq + 1] > sh.s_blo[qq])
-                        sh.s_contrib[k2++] = qq * 2 + (sh.s_blo[qq] >= pend_first[pi] ? 0 : 1);
+                sh.ep_ok = wait_bar_cluster(&sh.recvA[b], (uint32_t)((ua >> 1) & 1), limit_peer, &sh.abort, a.ctl,
+                                            kWaitPeers) ? 1 : 0;
+                if (sh.ep_ok) sh.pendA[b] = -1;
+                RS_TRACE_ONCE(kRtAReady);
             }
             named_bar_sync(1, 128);
-            const int r0 = rank * 128 / nc, r1 = (rank + 1) * 128 / nc, nrows = r1 - r0;
-            const int nitems = nrows * (N / 2);
-            const uint64_t t0 = globaltimer_ns();
-            for (int it = et; it < nitems && !failed; it += 128) {
-                const int rr = r0 + it % nrows, kp = it / nrows;
-                float sx = 0.f, sy = 0.f;
-                for (int c0 = 0; c0 < nc && !failed; c0 += 8) {
-                    const ulonglong2* src[8];
-                    ulonglong2 v[8];
+            if (!sh.ep_ok) { failed = true; break; }
+            // h = (k-half 0) + (k-half 1): two terms, and the sum does not depend on
+            // which block of the pair forms it
+            float z[NH];
+            {
+                const float4* rb = reinterpret_cast<const float4*>(recv + b * NH * 128) + row;
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        src[u] = partD + (size_t)sh.s_contrib[min(c0 + u, nc - 1)] * slot_pairs + kp * 128 + rr;
-                        v[u] = ld_relaxed_v2_b64(src[u]);
-                    }
-                    while (true) {   // re-read the pairs that are not this launch's yet (bounded)
-                        bool all = true;
+                for (int k4 = 0; k4 < NH / 4; ++k4) {
+                    const float4 pv = rb[k4 * 128];
+                    const float pw[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            if ((uint32_t)(v[u].x >> 32) != tag || (uint32_t)(v[u].y >> 32) != tag) {
-                                all = false;
-                                v[u] = ld_relaxed_v2_b64(src[u]);
-                            }
-                        if (all) break;
-                        if (sh.abort) { failed = true; break; }
-                        if (globaltimer_ns() - t0 > limit_peer) {
-                            record_error(a.ctl, kErrTimeout, kWaitPeers);
-                            sh.abort = 1;
-                            failed = true;
-                            break;
-                        }
-                    }
-                    if (failed) break;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (c0 + u < nc) {
-                            sx += __uint_as_float((uint32_t)v[u].x);
-                            sy += __uint_as_float((uint32_t)v[u].y);
-                        }
+                    for (int u = 0; u < 4; ++u)
+                        z[4 * k4 + u] = __uint_as_float(wk.hk ? r[NH + 4 * k4 + u] : r[4 * k4 + u]) + pw[u];
                 }
-                if (failed) break;
-                __nv_bfloat16* ycol = a.y + rt * 128 + rr;
-                if (2 * kp < nt) ycol[(size_t)(2 * kp) * a.d_h] = __float2bfloat16_rn(sx);
-                if (2 * kp + 1 < nt) ycol[(size_t)(2 * kp + 1) * a.d_h] = __float2bfloat16_rn(sy);
             }
-            if (et == 0) RS_TRACE_ONCE(kRtBReduced);
+            named_bar_sync(1, 128);
+            if (et == 0) {
+                RS_TRACE_ONCE(kRtARead);
+                // the peer may send into buffer b again (its unit ua + 2)
+                if (ua + 2 < wk.nA) mbar_arrive_relaxed_cluster(peer_freeA + (uint32_t)(b * 8));
+            }
+            // h' = bit ? g * Swish(h) : 0 (a select, so a masked token gives 0 even if
+            // its h is not finite), staged token-major in shared memory, then written
+            // with 16-byte stores: token t's 128 rows are 256 contiguous bytes
+            {
+                __nv_bfloat16* stg = hstage + row;
+#pragma unroll
+                for (int tl = 0; tl < NH; ++tl) {
+                    const float gsw = sh.s_gate[b][tg + tl] * rs_swish(z[tl]);
+                    stg[tl * 128] = __float2bfloat16_rn(((bits >> tl) & 1u) ? gsw : 0.f);
+                }
+            }
+            named_bar_sync(1, 128);
+            {
+                const uint4* src4 = reinterpret_cast<const uint4*>(hstage);
+                for (int c = et; c < NH * 16; c += 128) {
+                    const int tl = c >> 4, c16 = c & 15;
+                    uint4* dst4 =
+                        reinterpret_cast<uint4*>(a.hbuf + ((size_t)s * N + tg + tl) * a.d_e + mt * 128) + c16;
+                    *dst4 = src4[c];
+                }
+            }
+            // one release for the whole block: the barrier orders every thread's
+            // stores before thread 0's releasing count
+            named_bar_sync(1, 128);
+            if (et == 0) {
+                if ((v * 2 + wk.hk) != a.skip_unit) red_release_add_gpu(&readyA[s], 1u);
+                RS_TRACE_ONCE(kRtAWritten);
+            }
         }
         if (et == 0) {
-            RS_TRACE(kRtLastEpi);
-            // the peer may still read this block's last partial
-            if (nA > 0 && !failed)
-                wait_bar_cluster(&sh.part_free, (uint32_t)((nA - 1) & 1), limit_peer, &sh.abort, a.ctl, kWaitPeers);
+            RS_TRACE(kRtADone);
+            if (wk.nA > 0) mbar_arrive(&sh.a_pub);   // the producer may load expert-out tiles now
         }
+        // ---- expert-out row tiles: the cluster's 4 partials meet in shared memory
+        failed = failed || sh.abort;
+        if (doB) {
+            const uint32_t recv_u32 = smem_u32(recv);
+            for (int k = 0; k < wk.nRT && !failed; ++k) {
+                const int rt = wk.cid + k * wk.ncl;
+                const int ab = k & 1;
+                uint32_t r[32];
+                if (nBt > 0) {
+                    if (et == 0)
+                        sh.ep_ok = wait_bar(&sh.accB_full[ab], (uint32_t)((k >> 1) & 1), limit, &sh.abort, a.ctl,
+                                            kWaitAccFull) ? 1 : 0;
+                    named_bar_sync(1, 128);
+                    if (!sh.ep_ok) { failed = true; break; }
+                    tc_fence_after();
+                    const uint32_t taddr = tmem + ((uint32_t)(qd * 32) << 16) + accB_col + (uint32_t)(ab * N);
+                    if constexpr (N == 32) tmem_ld_32x32b_x32(taddr, r);
+                    else tmem_ld_32x32b_x16(taddr, r);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sh.accB_empty[ab]);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) r[t] = 0u;   // no tiles here: a zero contribution
+                }
+                if (k > 0) {
+                    // the receive area is reused: every other rank has summed the
+                    // quadrants this block sent it for the previous row tile
+                    if (et == 0)
+                        sh.ep_ok = wait_bar_cluster(&sh.freeB, (uint32_t)((k - 1) & 1), limit_peer, &sh.abort,
+                                                    a.ctl, kWaitPeers) ? 1 : 0;
+                    named_bar_sync(1, 128);
+                    if (!sh.ep_ok) { failed = true; break; }
+                }
+                if (qd != wk.cr) {
+                    // rows of quadrant qd are summed by rank qd: slot cr of its receive
+                    // area, [32 rows][N tokens] fp32
+                    const uint32_t dst = mapa_shared(recv_u32 + (uint32_t)((wk.cr * 32 + lane) * N * 4), (uint32_t)qd);
+                    const uint32_t rbar = mapa_shared(smem_u32(&sh.recvB), (uint32_t)qd);
+#pragma unroll
+                    for (int c4 = 0; c4 < N / 4; ++c4)
+                        st_async_v4(dst + (uint32_t)(c4 * 16), __uint_as_float(r[4 * c4]),
+                                    __uint_as_float(r[4 * c4 + 1]), __uint_as_float(r[4 * c4 + 2]),
+                                    __uint_as_float(r[4 * c4 + 3]), rbar);
+                    if (lane == 0) RS_TRACE_ONCE(kRtBSent);
+                } else {
+                    // this warp sums rows 32*cr .. 32*cr + 31 of the row tile over the 4
+                    // ranks, in rank order
+                    int ok = 1;
+                    if (lane == 0) {
+                        ok = wait_bar_cluster(&sh.recvB, (uint32_t)(k & 1), limit_peer, &sh.abort, a.ctl,
+                                              kWaitPeers) ? 1 : 0;
+                        if (ok) sh.pendB = -1;
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (ok) {
+                        float acc[N];
+#pragma unroll
+                        for (int t = 0; t < N; ++t) acc[t] = 0.f;
+#pragma unroll
+                        for (int q = 0; q < kRsCluster; ++q) {
+                            if (q == wk.cr) {
+#pragma unroll
+                                for (int t = 0; t < N; ++t) acc[t] += __uint_as_float(r[t]);
+                            } else {
+                                const float4* src = reinterpret_cast<const float4*>(recv + (q * 32 + lane) * N);
+#pragma unroll
+                                for (int c4 = 0; c4 < N / 4; ++c4) {
+                                    const float4 pv = src[c4];
+                                    acc[4 * c4] += pv.x;
+                                    acc[4 * c4 + 1] += pv.y;
+                                    acc[4 * c4 + 2] += pv.z;
+                                    acc[4 * c4 + 3] += pv.w;
+                                }
+                            }
+                        }
+                        // rows 32*cr.. of y for all tokens: staged [N tokens][32 rows]
+                        // bf16, then one TMA store (rows past T are clipped)
+                        if (k > 0 && lane == 0) bulk_wait_group_read0();   // staging free again
+                        __syncwarp();
+#pragma unroll
+                        for (int t = 0; t < N; ++t) hstage[t * 32 + lane] = __float2bfloat16_rn(acc[t]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_y, hstage, rt * 128 + wk.cr * 32, 0);
+                            bulk_commit_group();
+                            RS_TRACE_ONCE(kRtBReduced);
+                        }
+                    } else {
+                        failed = true;
+                    }
+                }
+                if (k + 1 < wk.nRT) {
+                    // hand the receive area back: re-arm it for the next row tile and
+                    // tell the other ranks this block has summed what they sent
+                    named_bar_sync(1, 128);
+                    if (et == 0 && !failed && !sh.abort) {
+                        mbar_arrive_expect_tx(&sh.recvB, 3u * 32u * N * 4u);
+                        sh.pendB = (k + 1) & 1;
+                        for (int q = 1; q < kRsCluster; ++q)
+                            mbar_arrive_relaxed_cluster(
+                                mapa_shared(smem_u32(&sh.freeB), (uint32_t)((wk.cr + q) % kRsCluster)));
+                    }
+                }
+            }
+        }
+        if (doB && qd == wk.cr && lane == 0) bulk_wait_group_read0();   // y's staging is read
+        if (et == 0) RS_TRACE(kRtLastEpi);
     }
 
     // --------------------------------------------------------------- teardown --
     __syncthreads();
+    if (threadIdx.x == 0) {
+        // a receive that was armed but never seen complete (a peer gave up or is
+        // late): give its bytes a bounded chance to land before this block leaves
+        for (int b = 0; b < 2; ++b)
+            if (sh.pendA[b] >= 0) wait_bar_drain(&sh.recvA[b], (uint32_t)sh.pendA[b], limit, a.ctl);
+        if (sh.pendB >= 0) wait_bar_drain(&sh.recvB, (uint32_t)sh.pendB, limit, a.ctl);
+    }
     if (warp == 2) {
-        if (lane == 0) wait_bar_drain(&sh.mma_done, 0, 2 * a.wait_ns, a.ctl);
+        if (lane == 0) wait_bar_drain(&sh.mma_done, 0, limit, a.ctl);
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kRsTmemCols);
     }
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const uint32_t old = atomicAdd(&a.ctl->done, 1u);
-        if (old == (uint32_t)(G - 1)) {
-            a.ctl->done = 0u;
-            atomicExch(&a.ctl->epoch, sh.epoch + 1u);
-        }
-        RS_TRACE(kRtEnd);
-    }
-    // no block leaves while its peer might still use its shared memory
-    cluster_barrier_sync();
+    if (threadIdx.x == 0) RS_TRACE(kRtEnd);
+    // no block leaves while a block of its cluster might still use its shared memory
+    cluster_barrier_sync_relaxed();
 }
 
 size_t forward_decode_smem_bytes() {
-    return 1024 + (size_t)kRsStages * kRsStageBytes + kRsPartBytes + kRsHStageBytes + sizeof(RsShared);
+    return 1024 + (size_t)kRsStages * kRsStageBytes + kRsRecvBytes + kRsHStageBytes + sizeof(RsShared);
 }
 
 template <int N>
-static cudaError_t launch_decode_n(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s,
-                                   bool cooperative) {
+static cudaError_t launch_decode_n(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s) {
     const size_t smem = forward_decode_smem_bytes();
     cudaError_t err =
         cudaFuncSetAttribute(union_expert_decode<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -768,38 +749,36 @@ static cudaError_t launch_decode_n(const DcArgs& a, const CUtensorMap* maps, int
     cfg.blockDim = dim3(kRsThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = kRsCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeCooperative;
-    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = cooperative ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, union_expert_decode<N>, maps[0], maps[1], maps[2], maps[3], a);
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, union_expert_decode<N>, maps[0], maps[1], maps[2], maps[3], maps[4], a);
 }
 
-cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s,
-                                  bool cooperative) {
-    if (a.N == 32) return launch_decode_n<32>(a, maps, grid, s, cooperative);
-    if (a.N == 16) return launch_decode_n<16>(a, maps, grid, s, cooperative);
+cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s) {
+    if (grid % kRsCluster != 0 || grid > kRsMaxG || a.E > kRsMaxE) return cudaErrorInvalidValue;
+    if (a.N == 32) return launch_decode_n<32>(a, maps, grid, s);
+    if (a.N == 16) return launch_decode_n<16>(a, maps, grid, s);
     return cudaErrorInvalidValue;
 }
 
-// Pairs of blocks (one block per SM) that can be resident at once, -1 on error.
-int decode_max_pairs() {
+// Clusters of 4 blocks (one block per SM) that can be resident at once, -1 on error.
+int decode_max_clusters() {
     const size_t smem = forward_decode_smem_bytes();
     if (cudaFuncSetAttribute(union_expert_decode<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return -1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2);
+    cfg.gridDim = dim3(kRsCluster);
     cfg.blockDim = dim3(kRsThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = kRsCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;

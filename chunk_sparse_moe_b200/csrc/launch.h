@@ -69,7 +69,6 @@ struct DcArgs {
     const float* gates;       // [T, E], T <= n
     __nv_bfloat16* y;         // [T, d_h]
     __nv_bfloat16* hbuf;      // [E slots][N][d_e] gated activations h'
-    unsigned long long* partD;  // [grid][2][N/2][128][2] expert-out partials, (launch tag << 32 | fp32 bits)
     uint32_t* readyA;         // [2][E] halves of an expert slot written, by launch parity
     Ctl* ctl;
     int T, d_h, E, d_e, n, N;
@@ -80,10 +79,12 @@ struct DcArgs {
     unsigned long long* trace;   // optional [grid][64] globaltimer stamps
 };
 // maps: x [T, d_h] (box N rows), W_in [E*d_e, d_h] and W_out [E*d_h, d_e] (box 128
-// rows), h' [E*N, d_e] (box N rows); all boxes 64 wide, 128-byte swizzle
-cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s,
-                                  bool cooperative);
+// rows), h' [E*N, d_e] (box N rows): boxes 64 wide, 128-byte swizzle; y [T, d_h]
+// (box 32 wide x N rows, no swizzle, for stores)
+cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s);
 size_t forward_decode_smem_bytes();
-int decode_max_pairs();
+// clusters of 4 blocks that can be resident at once (the launch uses 4 x this
+// many blocks), -1 on error
+int decode_max_clusters();
 
 }  // namespace bffn

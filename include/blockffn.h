@@ -158,16 +158,14 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
  *
  * Arguments as in blockffn_forward (x [T, d_h], gates [T, E] fp32, W_in, W_out,
  * y [T, d_h], device pointers owned by the caller); there is no workspace.  The
- * scratch is a fixed 16 MiB device array inside the library, which every GPU that
+ * scratch is a fixed 8 MiB device array inside the library, which every GPU that
  * loads the library holds until the process exits.  Shapes whose scratch would
- * exceed it (roughly E * d_e * 64 bytes plus 64 KB per SM) are rejected with
+ * exceed it (roughly E * d_e * 64 bytes) are rejected with
  * BLOCKFFN_ERR_UNSUPPORTED; so are T > n and non-bf16 data.  Nothing is
  * allocated: no cudaMalloc, cudaFree or allocating library call.
  * The first call on a device looks up the scratch's device address (with that
  * device current); make that first call before capturing any CUDA graph.  Every
- * call clears the scratch's status and counters on `stream` (all but its launch
- * counter, which tags each launch's partial sums and so must never repeat) and
- * then launches the forward.
+ * call clears the scratch's counters on `stream` and then launches the forward.
  * All calls share the one scratch array and it keeps the last call's contents:
  * calls that can overlap on the GPU (different streams, or concurrent host
  * threads) race and must not be issued.  Device-side timeouts are not reported
@@ -223,9 +221,9 @@ void blockffn_debug_skip_flag(int unit);
  * 5 last expert-in accumulator committed, 7 expert-in units finished, 8 first and
  * 9 last time every h' slot was seen ready, 10 last expert-out accumulator
  * committed, 11 last epilogue step, 13 end; for the block's first expert-in unit:
- * 14 accumulator read, 15 partial for the peer written, 16 peer's partial ready,
- * 17 peer's partial read, 18 h' published; 21 first expert-out partial stored,
- * 23 first slice of a split row tile summed, 24 first expert-out MMA issued.
+ * 14 accumulator read, 15 partial sent to the peer, 16 peer's partial received,
+ * 17 peer's partial read, 18 h' published; 21 first expert-out quadrant sent,
+ * 23 first 32 rows of y summed and stored, 24 first expert-out MMA issued.
  * Unset stamps stay 0.  NULL (the default) turns tracing off.
  */
 void blockffn_debug_set_trace(void* device_buffer);
