@@ -114,7 +114,12 @@ __device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t want, u
     }
 }
 
+// Named barrier over nthreads threads (whole warps).  The warp first gathers
+// all its lanes, so the aligned barrier is executed by a converged warp even
+// right after a branch that only one lane took (for instance lane 0 in a
+// bounded wait while lanes 1-31 went ahead).
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    __syncwarp();
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 

@@ -117,15 +117,16 @@ struct RingPos {
     }
 };
 
-// This block's expert-out tiles, in order: for each row tile rt = cid, cid +
-// #clusters, ... (< RT), the tiles j in [lo, hi) of that row tile, tile j being
-// expert slot j / KBe and 64-wide k-block j % KBe.  Stepped without divisions.
+// This block's expert-out tiles, in order: for each row tile rt = rt0, rt0 +
+// step, ... of its cluster, the tiles j in [lo, hi) of that row tile, tile j
+// being expert slot j / KBe and 64-wide k-block j % KBe.  Stepped without
+// divisions.
 struct BCursor {
     int rt, j, s, kb;
     int lo, hi, s0, kb0, step, KBe;
-    __device__ __forceinline__ void init(int cid, int ncl, int lo_, int hi_, int KBe_) {
-        rt = cid;
-        step = ncl;
+    __device__ __forceinline__ void init(int rt0, int rtstep, int lo_, int hi_, int KBe_) {
+        rt = rt0;
+        step = rtstep;
         lo = lo_;
         hi = hi_;
         KBe = KBe_;
@@ -152,7 +153,7 @@ struct BCursor {
 struct RsWork {
     int cr, cid, ncl, pr, hk;   // cluster rank, cluster, #clusters, pair, k-half
     int nA, apos, npairs;       // expert-in units of the pair: v = apos + u * npairs, u < nA
-    int nRT;                    // expert-out row tiles owned by the cluster
+    int nRT, rt0, rtstep;       // expert-out row tiles of the cluster: rt0, rt0 + rtstep, ...
     int bLo, bHi;               // this block's tiles of each of them
 };
 
@@ -164,15 +165,17 @@ __device__ __forceinline__ RsWork rs_work(int G, int P, int MT, int KBe, int RT)
     w.pr = w.cid * 2 + (w.cr >> 1);
     w.hk = w.cr & 1;
     w.npairs = 2 * w.ncl;
+    const int per_rt = P * KBe;
+    w.nRT = w.cid < RT ? (RT - w.cid + w.ncl - 1) / w.ncl : 0;
+    w.rt0 = w.cid;
+    w.rtstep = w.ncl;
+    w.bLo = per_rt * w.cr / kRsCluster;
+    w.bHi = per_rt * (w.cr + 1) / kRsCluster;
     // the A order: pairs of clusters without a row tile first
     const int nBc = min(RT, w.ncl);
     w.apos = w.pr >= 2 * nBc ? w.pr - 2 * nBc : w.pr + 2 * (w.ncl - nBc);
     const int VA = P * MT;
     w.nA = w.apos < VA ? (VA - w.apos + w.npairs - 1) / w.npairs : 0;
-    w.nRT = w.cid < RT ? (RT - w.cid + w.ncl - 1) / w.ncl : 0;
-    const int per_rt = P * KBe;
-    w.bLo = per_rt * w.cr / kRsCluster;
-    w.bHi = per_rt * (w.cr + 1) / kRsCluster;
     return w;
 }
 
@@ -321,13 +324,13 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             // Other blocks load at once and prefetch what the ring cannot hold yet.
             if (totB > 0) {
                 BCursor bc;
-                bc.init(wk.cid, wk.ncl, wk.bLo, wk.bHi, KBe);
+                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KBe);
                 for (int q = 0; q < totB; ++q, bc.advance())
                     if (wk.nA > 0 || q >= kRsStages)
                         tma_prefetch_l2_2d(&tm_wout, bc.kb * 64, sh.s_pair_e[bc.s] * a.d_h + bc.rt * 128);
                 if (wk.nA > 0 && !stop && !wait_bar(&sh.a_pub, 0u, limit, &sh.abort, a.ctl, kWaitEmpty))
                     stop = true;
-                bc.init(wk.cid, wk.ncl, wk.bLo, wk.bHi, KBe);
+                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KBe);
                 for (int q = 0; q < totB && !stop; ++q, ++i, rp.advance(), bc.advance()) {
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
                         stop = true;
@@ -442,9 +445,12 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 done = __all_sync(0xffffffffu, mine_ok);
                 if (done) break;
                 __nanosleep(64);
-                if (__any_sync(0xffffffffu, sh.abort != 0)) break;
-                if (globaltimer_ns() - t0 > limit_peer) {
-                    if (lane == 0) {
+                // the whole warp gives up together: lane 0's clock decides the
+                // timeout (lanes read the clock at slightly different times)
+                const bool aborted = __any_sync(0xffffffffu, sh.abort != 0);
+                const bool timed_out = __shfl_sync(0xffffffffu, globaltimer_ns() - t0 > limit_peer ? 1 : 0, 0) != 0;
+                if (aborted || timed_out) {
+                    if (lane == 0 && !aborted) {
                         record_error(a.ctl, kErrTimeout, kWaitFlag);
                         sh.abort = 1;
                     }
@@ -460,7 +466,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 RS_TRACE(kRtLastFlag);
                 const uint64_t pol = policy_evict_first();
                 BCursor bc;
-                bc.init(wk.cid, wk.ncl, wk.bLo, wk.bHi, KBe);
+                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KBe);
                 for (int q = 0; q < totB; ++q, ++i, rp.advance(), bc.advance()) {
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) break;
                     mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 128));
@@ -607,7 +613,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         if (doB) {
             const uint32_t recv_u32 = smem_u32(recv);
             for (int k = 0; k < wk.nRT && !failed; ++k) {
-                const int rt = wk.cid + k * wk.ncl;
+                const int rt = wk.rt0 + k * wk.rtstep;
                 const int ab = k & 1;
                 uint32_t r[32];
                 if (nBt > 0) {
@@ -715,6 +721,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     }
 
     // --------------------------------------------------------------- teardown --
+    __syncwarp();
     __syncthreads();
     if (threadIdx.x == 0) {
         // a receive that was armed but never seen complete (a peer gave up or is

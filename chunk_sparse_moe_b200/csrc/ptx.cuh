@@ -125,6 +125,15 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// relaxed atomic add / load at GPU scope: counters that order no data
+__device__ __forceinline__ void red_relaxed_add_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 // atomic add with release semantics at GPU scope: writes this thread has made or
 // observed (through a barrier) before it are visible to whoever acquires the count
 __device__ __forceinline__ void red_release_add_gpu(uint32_t* p, uint32_t v) {
@@ -305,7 +314,9 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
     return v;
 }
+// (aligned forms, so each warp gathers its lanes first)
 __device__ __forceinline__ void cluster_barrier_sync() {
+    __syncwarp();
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
 }
@@ -313,6 +324,7 @@ __device__ __forceinline__ void cluster_barrier_sync() {
 // the cluster may still touch its shared memory", where every such access is
 // already accounted for by an mbarrier wait
 __device__ __forceinline__ void cluster_barrier_sync_relaxed() {
+    __syncwarp();
     asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
