@@ -56,7 +56,7 @@ constexpr int kRsMaxE = 256;
 constexpr int kRsMaxG = 160;
 // receive area: two expert-in partials for this block's half of the tokens
 // ([<=16 tokens][128 rows] fp32 each); later the expert-out quadrant partials
-// from the other 3 ranks ([4 slots][32 rows][<=32 tokens] fp32) reuse it
+// from the other 3 ranks ([4 slots][<=32 tokens][32 rows] fp32) reuse it
 constexpr int kRsRecvBytes = 2 * 16 * 128 * 4;
 constexpr int kRsHStageBytes = 16 * 128 * 2;  // this block's half of h' [<=16 tokens][128 rows] bf16
 static_assert(4 * 32 * 32 * 4 <= kRsRecvBytes, "expert-out quadrants fit the receive area");
@@ -645,12 +645,14 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 }
                 if (qd != wk.cr) {
                     // rows of quadrant qd are summed by rank qd: slot cr of its receive
-                    // area, [32 rows][N tokens] fp32
-                    const uint32_t dst = mapa_shared(recv_u32 + (uint32_t)((wk.cr * 32 + lane) * N * 4), (uint32_t)qd);
+                    // area, float4 of tokens 4c..4c+3 of a row at [c][row] (consecutive
+                    // lanes, consecutive 16 bytes: no bank conflicts on either side)
+                    const uint32_t dst =
+                        mapa_shared(recv_u32 + (uint32_t)((wk.cr * (N / 4) * 32 + lane) * 16), (uint32_t)qd);
                     const uint32_t rbar = mapa_shared(smem_u32(&sh.recvB), (uint32_t)qd);
 #pragma unroll
                     for (int c4 = 0; c4 < N / 4; ++c4)
-                        st_async_v4(dst + (uint32_t)(c4 * 16), __uint_as_float(r[4 * c4]),
+                        st_async_v4(dst + (uint32_t)(c4 * 32 * 16), __uint_as_float(r[4 * c4]),
                                     __uint_as_float(r[4 * c4 + 1]), __uint_as_float(r[4 * c4 + 2]),
                                     __uint_as_float(r[4 * c4 + 3]), rbar);
                     if (lane == 0) RS_TRACE_ONCE(kRtBSent);
@@ -674,10 +676,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
 #pragma unroll
                                 for (int t = 0; t < N; ++t) acc[t] += __uint_as_float(r[t]);
                             } else {
-                                const float4* src = reinterpret_cast<const float4*>(recv + (q * 32 + lane) * N);
+                                const float4* src = reinterpret_cast<const float4*>(recv) + q * (N / 4) * 32 + lane;
 #pragma unroll
                                 for (int c4 = 0; c4 < N / 4; ++c4) {
-                                    const float4 pv = src[c4];
+                                    const float4 pv = src[c4 * 32];
                                     acc[4 * c4] += pv.x;
                                     acc[4 * c4 + 1] += pv.y;
                                     acc[4 * c4 + 2] += pv.z;
