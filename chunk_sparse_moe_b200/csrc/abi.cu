@@ -79,6 +79,24 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A bf16 matrix [rows, cols] (cols contiguous, row pitch cols*2 bytes) seen as a
+// 3-D tensor {64-wide column block element, row, column block}: a box {64,
+// box_rows, 2} fetches two consecutive 64-column blocks of box_rows rows and
+// lands as two [box_rows x 128 B] 128-byte-swizzled tiles, one after the other.
+// One TMA operation instead of two: the per-operation cost dominates below
+// ~32 KB.  cols must be a multiple of 128.
+bool make_map_kpair(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr || cols % 128 != 0) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor [outer, inner], box {box_inner, box_outer}, no swizzle (for
 // tiled stores from a plain row-major shared-memory tile).
 bool make_map_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -298,15 +316,15 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         ncl = clusters_cache[dev_id];
         if (ncl > G / 4) ncl = G / 4;
     }
-    if (fuse && ncl > 0 && 4 * ncl <= 160 && L.KB % 2 == 0 && E <= 256) {
+    if (fuse && ncl > 0 && 4 * ncl <= 160 && L.KB % 4 == 0 && E <= 256) {
         // one chunk: clusters of 4 blocks, expert-in in k-half pairs, expert-out
         // row tiles summed inside the cluster (forward_decode.cu)
         const int Gd = 4 * ncl;
         CUtensorMap dmaps[5];
-        if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
-            !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
-            !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
-            !make_map(&dmaps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)E * L.N, (uint32_t)L.N) ||
+        if (!make_map_kpair(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
+            !make_map_kpair(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
+            !make_map_kpair(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
+            !make_map_kpair(&dmaps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)E * L.N, (uint32_t)L.N) ||
             !make_map_plain(&dmaps[4], y, (uint64_t)d_h, (uint64_t)T, 32, (uint32_t)L.N))
             return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
         DcArgs da;
@@ -426,7 +444,7 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     std::call_once(clusters_once[dev], [&]() { clusters_cache[dev] = decode_max_clusters(); });
     int ncl = clusters_cache[dev];
     if (ncl > G / 4) ncl = G / 4;
-    if (ncl <= 0 || 4 * ncl > 160 || (d_h / 64) % 2 != 0 || E > 256)
+    if (ncl <= 0 || 4 * ncl > 160 || (d_h / 64) % 4 != 0 || E > 256)
         return fail(BLOCKFFN_ERR_UNSUPPORTED, "no-allocation forward: single-chunk kernel unavailable here");
     const int Gd = 4 * ncl;
     const int N = n <= 16 ? 16 : 32;
@@ -449,10 +467,10 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     e = cudaMemsetAsync(scratch, 0, zero_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "no-allocation scratch clear");
     CUtensorMap dmaps[5];
-    if (!make_map(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)N) ||
-        !make_map(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
-        !make_map(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
-        !make_map(&dmaps[3], scratch + off_h, (uint64_t)d_e, (uint64_t)E * N, (uint32_t)N) ||
+    if (!make_map_kpair(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)N) ||
+        !make_map_kpair(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
+        !make_map_kpair(&dmaps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
+        !make_map_kpair(&dmaps[3], scratch + off_h, (uint64_t)d_e, (uint64_t)E * N, (uint32_t)N) ||
         !make_map_plain(&dmaps[4], y, (uint64_t)d_h, (uint64_t)T, 32, (uint32_t)N))
         return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     DcArgs da;

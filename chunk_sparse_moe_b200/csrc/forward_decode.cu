@@ -16,7 +16,7 @@
 // (d_e = 128: the whole expert).  The pair at position p of the A order takes
 // units p, p + #pairs, ...; its block of rank r in the pair multiplies the
 // k-half r of W_in_e (tcgen05; weights as the M = 128 operand, the chunk's N
-// tokens as N) into a TMEM accumulator.  The two blocks split the tokens: each
+// tokens as N) into a TMEM accumulator, two 64-wide k-blocks per pipeline stage.  The two blocks split the tokens: each
 // sends the peer its partial for the peer's half with st.async straight into
 // the peer's shared memory (the bytes are counted on the peer's mbarrier), adds
 // the peer's partial for its own half, applies the post-hoc mask, the gate and
@@ -26,8 +26,8 @@
 //
 // Expert-out (B).  y^T = sum_e W_out_e h'_e^T with W_out_e's 128-row tiles as the
 // M operand and the tokens as N.  Cluster c owns the row tiles c, c + #clusters,
-// ...; each of its 4 blocks takes a quarter of a row tile's (expert, 64-wide
-// k-block) tiles.  A tile waits (bounded) until every expert's h' is counted
+// ...; each of its 4 blocks takes a quarter of a row tile's (expert, pair of
+// 64-wide k-blocks) tiles.  A tile waits (bounded) until every expert's h' is counted
 // in, then its h' slice arrives by TMA.  The 4 partial tiles are summed inside
 // the cluster: warp q of every block st.async's its 32 accumulator rows to the
 // block of rank q, which adds the 4 contributions in rank order (a fixed order)
@@ -49,8 +49,13 @@ namespace bffn {
 
 constexpr int kRsThreads = 224;
 constexpr int kRsCluster = 4;
-constexpr int kRsStages = 10;
-constexpr int kRsStageBytes = 16384 + 4096;  // weight tile [128 x 64] + activation tile [<=32 x 64]
+constexpr int kRsStages = 5;
+// a stage: weight tile [128 rows x 128] + activation tile [<=32 rows x 128], each
+// as two 64-wide k-blocks of 128-byte-swizzled rows, each fetched by one 3-D TMA
+// operation (a TMA operation costs about the same below ~32 KB, so fewer and
+// larger ones move more bytes per SM)
+constexpr int kRsWBytes = 32768;
+constexpr int kRsStageBytes = kRsWBytes + 8192;
 constexpr int kRsTmemCols = 128;             // 2 expert-in + 2 expert-out accumulators of <=32 columns
 constexpr int kRsMaxE = 256;
 constexpr int kRsMaxG = 160;
@@ -119,19 +124,19 @@ struct RingPos {
 
 // This block's expert-out tiles, in order: for each row tile rt = rt0, rt0 +
 // step, ... of its cluster, the tiles j in [lo, hi) of that row tile, tile j
-// being expert slot j / KBe and 64-wide k-block j % KBe.  Stepped without
-// divisions.
+// being expert slot j / KPe and pair of 64-wide k-blocks kb = j % KPe (k-blocks
+// 2kb and 2kb+1).  Stepped without divisions.
 struct BCursor {
     int rt, j, s, kb;
-    int lo, hi, s0, kb0, step, KBe;
-    __device__ __forceinline__ void init(int rt0, int rtstep, int lo_, int hi_, int KBe_) {
+    int lo, hi, s0, kb0, step, KPe;
+    __device__ __forceinline__ void init(int rt0, int rtstep, int lo_, int hi_, int KPe_) {
         rt = rt0;
         step = rtstep;
         lo = lo_;
         hi = hi_;
-        KBe = KBe_;
-        s0 = lo / KBe;
-        kb0 = lo - s0 * KBe;
+        KPe = KPe_;
+        s0 = lo / KPe;
+        kb0 = lo - s0 * KPe;
         j = lo;
         s = s0;
         kb = kb0;
@@ -142,7 +147,7 @@ struct BCursor {
             s = s0;
             kb = kb0;
             rt += step;
-        } else if (++kb == KBe) {
+        } else if (++kb == KPe) {
             kb = 0;
             ++s;
         }
@@ -157,7 +162,7 @@ struct RsWork {
     int bLo, bHi;               // this block's tiles of each of them
 };
 
-__device__ __forceinline__ RsWork rs_work(int G, int P, int MT, int KBe, int RT) {
+__device__ __forceinline__ RsWork rs_work(int G, int P, int MT, int KPe, int RT) {
     RsWork w;
     w.cr = (int)cluster_ctarank();
     w.cid = (int)blockIdx.x / kRsCluster;
@@ -165,7 +170,7 @@ __device__ __forceinline__ RsWork rs_work(int G, int P, int MT, int KBe, int RT)
     w.pr = w.cid * 2 + (w.cr >> 1);
     w.hk = w.cr & 1;
     w.npairs = 2 * w.ncl;
-    const int per_rt = P * KBe;
+    const int per_rt = P * KPe;
     w.nRT = w.cid < RT ? (RT - w.cid + w.ncl - 1) / w.ncl : 0;
     w.rt0 = w.cid;
     w.rtstep = w.ncl;
@@ -193,9 +198,9 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     RsShared& sh = *reinterpret_cast<RsShared*>(smem + kRsStages * kRsStageBytes + kRsRecvBytes + kRsHStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
-    const int KBe = a.d_e / 64;     // 64-wide k-blocks of one expert in the expert-out GEMM
+    const int KPe = a.d_e / 128;    // k-block pairs of one expert in the expert-out GEMM
     const int MT = a.d_e / 128;     // 128-row tiles of W_in_e
-    const int KBh = a.KB / 2;       // k-tiles of one k-half
+    const int KP = a.KB / 4;        // k-block pairs of one k-half in the expert-in GEMM
     const int nt = min(a.n, a.T);
 
     if (threadIdx.x == 0) {
@@ -274,7 +279,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     __syncthreads();
     tc_fence_after();
     const int P = sh.P;
-    const RsWork wk = rs_work(G, P, MT, KBe, a.RT);
+    const RsWork wk = rs_work(G, P, MT, KPe, a.RT);
     const int nBt = wk.bHi - wk.bLo;                 // expert-out tiles per owned row tile
     const int totB = P > 0 ? wk.nRT * nBt : 0;        // this block's expert-out tiles
     const bool doB = P > 0 && wk.nRT > 0;             // this cluster sums expert-out row tiles
@@ -304,16 +309,16 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             for (int ua = 0; ua < wk.nA && !stop; ++ua) {
                 const int v = wk.apos + ua * wk.npairs;
                 const int e = sh.s_pair_e[v / MT], mt = v % MT;
-                for (int t = 0; t < KBh; ++t, ++i, rp.advance()) {
-                    const int kt = wk.hk * KBh + t;
+                for (int t = 0; t < KP; ++t, ++i, rp.advance()) {
+                    const int kb = 2 * (wk.hk * KP + t);   // first of the stage's two k-blocks
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
                         stop = true;
                         break;
                     }
                     uint8_t* w = smem + rp.st * kRsStageBytes;
-                    mbar_arrive_expect_tx(&sh.full_w[rp.st], 16384 + N * 128);
-                    tma_load_2d(w, &tm_win, &sh.full_w[rp.st], kt * 64, e * a.d_e + mt * 128, pol_stream);
-                    tma_load_2d(w + 16384, &tm_x, &sh.full_w[rp.st], kt * 64, 0, pol_keep);
+                    mbar_arrive_expect_tx(&sh.full_w[rp.st], kRsWBytes + N * 256);
+                    tma_load_3d(w, &tm_win, &sh.full_w[rp.st], 0, e * a.d_e + mt * 128, kb, pol_stream);
+                    tma_load_3d(w + kRsWBytes, &tm_x, &sh.full_w[rp.st], 0, 0, kb, pol_keep);
                     if (i == 0) RS_TRACE(kRtFirstLoad);
                 }
             }
@@ -324,21 +329,21 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             // Other blocks load at once and prefetch what the ring cannot hold yet.
             if (totB > 0) {
                 BCursor bc;
-                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KBe);
+                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
                 for (int q = 0; q < totB; ++q, bc.advance())
                     if (wk.nA > 0 || q >= kRsStages)
-                        tma_prefetch_l2_2d(&tm_wout, bc.kb * 64, sh.s_pair_e[bc.s] * a.d_h + bc.rt * 128);
+                        tma_prefetch_l2_3d(&tm_wout, 0, sh.s_pair_e[bc.s] * a.d_h + bc.rt * 128, 2 * bc.kb);
                 if (wk.nA > 0 && !stop && !wait_bar(&sh.a_pub, 0u, limit, &sh.abort, a.ctl, kWaitEmpty))
                     stop = true;
-                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KBe);
+                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
                 for (int q = 0; q < totB && !stop; ++q, ++i, rp.advance(), bc.advance()) {
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
                         stop = true;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sh.full_w[rp.st], 16384);
-                    tma_load_2d(smem + rp.st * kRsStageBytes, &tm_wout, &sh.full_w[rp.st], bc.kb * 64,
-                                sh.s_pair_e[bc.s] * a.d_h + bc.rt * 128, pol_stream);
+                    mbar_arrive_expect_tx(&sh.full_w[rp.st], kRsWBytes);
+                    tma_load_3d(smem + rp.st * kRsStageBytes, &tm_wout, &sh.full_w[rp.st], 0,
+                                sh.s_pair_e[bc.s] * a.d_h + bc.rt * 128, 2 * bc.kb, pol_stream);
                     if (i == 0) RS_TRACE(kRtFirstLoad);
                 }
             }
@@ -360,7 +365,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem + accA_col + (uint32_t)(ab * N);
-                for (int t = 0; t < KBh; ++t, ++i, rp.advance()) {
+                for (int t = 0; t < KP; ++t, ++i, rp.advance()) {
                     const int st = rp.st;
                     if (!wait_bar(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
                         !wait_bar(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
@@ -370,11 +375,14 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     tc_fence_after();
                     if (i == 0) RS_TRACE(kRtFirstFull);
                     const uint32_t wb = smem_u32(smem + st * kRsStageBytes);
-                    const uint32_t xb = wb + 16384;
+                    const uint32_t xb = wb + kRsWBytes;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(d, sw128_kmajor_desc(wb + kk * 32), sw128_kmajor_desc(xb + kk * 32), idesc,
-                                  (t > 0 || kk > 0) ? 1u : 0u);
+                    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d, sw128_kmajor_desc(wb + kb * 16384 + kk * 32),
+                                      sw128_kmajor_desc(xb + kb * N * 128 + kk * 32), idesc,
+                                      (t > 0 || kb > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sh.empty[st]);
                 }
                 if (stop) break;
@@ -399,11 +407,14 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     tc_fence_after();
                     if (k == 0 && q == 0) RS_TRACE(kRtFirstBMma);
                     const uint32_t wb = smem_u32(smem + st * kRsStageBytes);
-                    const uint32_t hb = wb + 16384;
+                    const uint32_t hb = wb + kRsWBytes;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(d, sw128_kmajor_desc(wb + kk * 32), sw128_kmajor_desc(hb + kk * 32), idesc,
-                                  (q > 0 || kk > 0) ? 1u : 0u);
+                    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d, sw128_kmajor_desc(wb + kb * 16384 + kk * 32),
+                                      sw128_kmajor_desc(hb + kb * N * 128 + kk * 32), idesc,
+                                      (q > 0 || kb > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&sh.empty[st]);
                 }
                 if (stop) break;
@@ -418,7 +429,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // tile the warp waits (bounded) until every expert slot's h' is counted in;
         // then lane 0 moves each tile's [N x 64] h' slice with one TMA load, which
         // lands in the same 128-byte-swizzled layout as the weight tile's operand.
-        const long long nAt = (long long)wk.nA * KBh;
+        const long long nAt = (long long)wk.nA * KP;
         long long i = 0;
         RingPos rp;
         int stop = sh.abort != 0;
@@ -466,12 +477,12 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 RS_TRACE(kRtLastFlag);
                 const uint64_t pol = policy_evict_first();
                 BCursor bc;
-                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KBe);
+                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
                 for (int q = 0; q < totB; ++q, ++i, rp.advance(), bc.advance()) {
                     if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) break;
-                    mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 128));
-                    tma_load_2d(smem + rp.st * kRsStageBytes + 16384, &tm_h, &sh.full_h[rp.st], bc.kb * 64,
-                                bc.s * N, pol);
+                    mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 256));
+                    tma_load_3d(smem + rp.st * kRsStageBytes + kRsWBytes, &tm_h, &sh.full_h[rp.st], 0, bc.s * N,
+                                2 * bc.kb, pol);
                 }
                 // no copy into this block's shared memory outlives it
                 for (long long q = i - kRsStages < nAt ? nAt : i - kRsStages; q < i; ++q)

@@ -79,8 +79,9 @@ struct DcArgs {
     unsigned long long* trace;   // optional [grid][64] globaltimer stamps
 };
 // maps: x [T, d_h] (box N rows), W_in [E*d_e, d_h] and W_out [E*d_h, d_e] (box 128
-// rows), h' [E*N, d_e] (box N rows): boxes 64 wide, 128-byte swizzle; y [T, d_h]
-// (box 32 wide x N rows, no swizzle, for stores)
+// rows), h' [E*N, d_e] (box N rows): 3-D {64, rows, column block} boxes of two
+// 64-wide column blocks, 128-byte swizzle; y [T, d_h] (box 32 wide x N rows, no
+// swizzle, for stores)
 cudaError_t launch_forward_decode(const DcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s);
 size_t forward_decode_smem_bytes();
 // clusters of 4 blocks that can be resident at once (the launch uses 4 x this
