@@ -38,7 +38,8 @@ struct Ctl {
     int32_t detail;        // which wait / check
     uint32_t epoch;        // number of completed forward launches (flag stamp)
     uint32_t done;         // thread blocks of the current launch that finished
-    uint32_t pad[60];
+    uint32_t issued[2];    // by launch parity: blocks that issued their last expert-in load
+    uint32_t pad[58];
 };
 static_assert(sizeof(Ctl) == 256, "control block is 256 bytes");
 

@@ -228,6 +228,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const int32_t st0 = __ldcg(&a.ctl->status);
         // acquire: the read is done before this block's count below is seen
         const uint32_t ep0 = ld_acquire_gpu(&a.ctl->epoch);
+        if (blockIdx.x == 0) a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;   // the next launch's counter
         sh.abort = st0 != 0;
         sh.epoch = ep0;
         // The last block to read the launch counter advances it for the next
@@ -322,11 +323,22 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     if (i == 0) RS_TRACE(kRtFirstLoad);
                 }
             }
+            if (wk.nA > 0) red_relaxed_add_gpu(&a.ctl->issued[par], 1u);
             // Expert-out weights.  A block with expert-in units sends all of its
             // tiles towards L2 now and loads them into the ring only after its h'
             // is published: a release waits for the block's bulk loads in flight,
             // and no expert-out MMA can start before every h' is out anyway.
-            // Other blocks load at once and prefetch what the ring cannot hold yet.
+            // Other blocks first let every expert-in block issue its last load (a
+            // scheduling hint, bounded and never an error: their requests then
+            // queue behind the expert-in weights, which are on the critical path),
+            // then load and prefetch what the ring cannot hold yet.
+            if (totB > 0 && wk.nA == 0 && !stop) {
+                const uint32_t nAblocks = 2u * (uint32_t)min(P * MT, wk.npairs);
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_relaxed_gpu(&a.ctl->issued[par]) < nAblocks && globaltimer_ns() - t0 < 20000ull &&
+                       !sh.abort)
+                    __nanosleep(64);
+            }
             if (totB > 0) {
                 BCursor bc;
                 bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
