@@ -65,6 +65,32 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_
     }
 }
 
+// The same wait made by all 32 lanes of a warp together, with one outcome for
+// the whole warp (lane 0's observations decide), so the warp's control flow stays
+// uniform: a role whose loop runs on every lane and issues through one elected
+// lane keeps its instructions flowing at the converged rate, where a loop run by
+// one lane alone while the others wait was measured to issue tcgen05 work at
+// about half that rate.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                              volatile int* abort, Ctl* ctl, int32_t detail) {
+    if (__shfl_sync(0xffffffffu, mbar_try_wait(bar, parity) ? 1 : 0, 0)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        int st = mbar_try_wait(bar, parity) ? 1 : (*abort ? 2 : (globaltimer_ns() - t0 > limit_ns ? 3 : 0));
+        st = __shfl_sync(0xffffffffu, st, 0);
+        if (st == 1) return true;
+        if (st == 2) return false;
+        if (st == 3) {
+            if ((threadIdx.x & 31) == 0) {
+                record_error(ctl, kErrTimeout, detail);
+                *abort = 1;
+            }
+            __syncwarp();
+            return false;
+        }
+    }
+}
+
 // Same, acquiring at cluster scope (for barriers that blocks of the cluster
 // arrive on remotely).
 __device__ __forceinline__ bool wait_bar_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns,

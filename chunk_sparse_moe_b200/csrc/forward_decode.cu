@@ -122,6 +122,23 @@ struct RingPos {
     }
 };
 
+// The 8 MMAs of one pipeline stage: D (+)= W[128 x 128] * act[N x 128]^T, the
+// weight tile at the stage's start and the activation tile after it, each as two
+// 64-wide k-blocks in the 128-byte-swizzled K-major layout TMA writes.  ds is the
+// descriptor of the stage's first byte; every operand's descriptor is ds plus a
+// compile-time offset (computing each one from a run-time address made the
+// issuing thread markedly slower per stage than the tensor core).
+template <int N>
+__device__ __forceinline__ void rs_stage_mma(uint32_t d, uint64_t ds, uint32_t idesc, bool acc) {
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(d, ds + (uint64_t)((kb * 16384 + kk * 32) >> 4),
+                      ds + (uint64_t)((kRsWBytes + kb * N * 128 + kk * 32) >> 4), idesc,
+                      (acc || kb > 0 || kk > 0) ? 1u : 0u);
+}
+
 // This block's expert-out tiles, in order: for each row tile rt = rt0, rt0 +
 // step, ... of its cluster, the tiles j in [lo, hi) of that row tile, tile j
 // being expert slot j / KPe and pair of 64-wide k-blocks kb = j % KPe (k-blocks
@@ -365,76 +382,96 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer --
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, N);     // 128 weight rows x tokens
-            long long i = 0;
-            RingPos rp;
-            bool stop = sh.abort != 0;
-            for (int ua = 0; ua < wk.nA && !stop; ++ua) {
-                const int ab = ua & 1;
-                if (!wait_bar(&sh.accA_empty[ab], (uint32_t)(((ua >> 1) & 1) ^ 1), limit, &sh.abort, a.ctl,
-                              kWaitAccEmpty))
+        // The whole warp runs the loops with warp-wide waits; one elected lane
+        // issues the MMAs and commits.
+        const bool leader = elect_one();
+        const uint32_t idesc = idesc_bf16_f32(128, N);     // 128 weight rows x tokens
+        // shared addresses are below 2^18, so stage offsets added to the
+        // descriptor's start-address field never carry out of it
+        const uint64_t desc0 = sw128_kmajor_desc(smem_u32(smem));
+        long long i = 0;
+        RingPos rp;
+        bool stop = __shfl_sync(0xffffffffu, sh.abort, 0) != 0;
+        // the current ring position's barriers as last tested (a stale "not yet"
+        // only costs a blocking wait)
+        uint32_t rw = 0u, rh = 0u;
+        for (int ua = 0; ua < wk.nA && !stop; ++ua) {
+            const int ab = ua & 1;
+            if (!wait_bar_warp(&sh.accA_empty[ab], (uint32_t)(((ua >> 1) & 1) ^ 1), limit, &sh.abort, a.ctl,
+                               kWaitAccEmpty))
+                break;
+            tc_fence_after();
+            const uint32_t d = tmem + accA_col + (uint32_t)(ab * N);
+            for (int t = 0; t < KP; ++t, ++i, rp.advance()) {
+                const int st = rp.st;
+                if (!__all_sync(0xffffffffu, rw & rh) &&
+                    (!wait_bar_warp(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
+                     !wait_bar_warp(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH))) {
+                    stop = true;
                     break;
+                }
                 tc_fence_after();
-                const uint32_t d = tmem + accA_col + (uint32_t)(ab * N);
-                for (int t = 0; t < KP; ++t, ++i, rp.advance()) {
-                    const int st = rp.st;
-                    if (!wait_bar(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
-                        !wait_bar(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
-                        stop = true;
-                        break;
-                    }
-                    tc_fence_after();
+                {
+                    // test the next ring position now: the two shared-memory round
+                    // trips then overlap this stage's MMAs instead of preceding the next
+                    RingPos nx = rp;
+                    nx.advance();
+                    rw = mbar_test_wait(&sh.full_w[nx.st], nx.ph);
+                    rh = mbar_test_wait(&sh.full_h[nx.st], nx.ph);
+                }
+                if (leader) {
                     if (i == 0) RS_TRACE(kRtFirstFull);
-                    const uint32_t wb = smem_u32(smem + st * kRsStageBytes);
-                    const uint32_t xb = wb + kRsWBytes;
-#pragma unroll
-                    for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(d, sw128_kmajor_desc(wb + kb * 16384 + kk * 32),
-                                      sw128_kmajor_desc(xb + kb * N * 128 + kk * 32), idesc,
-                                      (t > 0 || kb > 0 || kk > 0) ? 1u : 0u);
+                    rs_stage_mma<N>(d, desc0 + (uint64_t)(st * (kRsStageBytes >> 4)), idesc, t > 0);
                     umma_commit(&sh.empty[st]);
                 }
-                if (stop) break;
+                __syncwarp();
+            }
+            if (stop) break;
+            if (leader) {
                 umma_commit(&sh.accA_full[ab]);
                 RS_TRACE(kRtLastACommit);
             }
-            // one accumulator per owned row tile, alternating between two
-            for (int k = 0; k < (totB > 0 ? wk.nRT : 0) && !stop; ++k) {
-                const int ab = k & 1;
-                if (!wait_bar(&sh.accB_empty[ab], (uint32_t)(((k >> 1) & 1) ^ 1), limit, &sh.abort, a.ctl,
-                              kWaitAccEmpty))
+            __syncwarp();
+        }
+        // one accumulator per owned row tile, alternating between two
+        for (int k = 0; k < (totB > 0 ? wk.nRT : 0) && !stop; ++k) {
+            const int ab = k & 1;
+            if (!wait_bar_warp(&sh.accB_empty[ab], (uint32_t)(((k >> 1) & 1) ^ 1), limit, &sh.abort, a.ctl,
+                               kWaitAccEmpty))
+                break;
+            tc_fence_after();
+            const uint32_t d = tmem + accB_col + (uint32_t)(ab * N);
+            for (int q = 0; q < nBt; ++q, ++i, rp.advance()) {
+                const int st = rp.st;
+                if (!__all_sync(0xffffffffu, rw & rh) &&
+                    (!wait_bar_warp(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
+                     !wait_bar_warp(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH))) {
+                    stop = true;
                     break;
+                }
                 tc_fence_after();
-                const uint32_t d = tmem + accB_col + (uint32_t)(ab * N);
-                for (int q = 0; q < nBt; ++q, ++i, rp.advance()) {
-                    const int st = rp.st;
-                    if (!wait_bar(&sh.full_w[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
-                        !wait_bar(&sh.full_h[st], rp.ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
-                        stop = true;
-                        break;
-                    }
-                    tc_fence_after();
+                {
+                    RingPos nx = rp;
+                    nx.advance();
+                    rw = mbar_test_wait(&sh.full_w[nx.st], nx.ph);
+                    rh = mbar_test_wait(&sh.full_h[nx.st], nx.ph);
+                }
+                if (leader) {
                     if (k == 0 && q == 0) RS_TRACE(kRtFirstBMma);
-                    const uint32_t wb = smem_u32(smem + st * kRsStageBytes);
-                    const uint32_t hb = wb + kRsWBytes;
-#pragma unroll
-                    for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(d, sw128_kmajor_desc(wb + kb * 16384 + kk * 32),
-                                      sw128_kmajor_desc(hb + kb * N * 128 + kk * 32), idesc,
-                                      (q > 0 || kb > 0 || kk > 0) ? 1u : 0u);
+                    rs_stage_mma<N>(d, desc0 + (uint64_t)(st * (kRsStageBytes >> 4)), idesc, q > 0);
                     umma_commit(&sh.empty[st]);
                 }
-                if (stop) break;
+                __syncwarp();
+            }
+            if (stop) break;
+            if (leader) {
                 umma_commit(&sh.accB_full[ab]);
                 RS_TRACE(kRtLastCommit);
             }
-            umma_commit(&sh.mma_done);
+            __syncwarp();
         }
+        if (leader) umma_commit(&sh.mma_done);
+        __syncwarp();
     } else if (warp == 2) {
         // ------------------------------------------------------- h' loader --
         // A stages carry no h': lane 0 just arrives.  Before the first expert-out
