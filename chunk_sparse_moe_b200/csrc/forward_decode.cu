@@ -306,7 +306,12 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         mbar_arrive_expect_tx(&sh.recvB, 3u * 32u * N * 4u);
         sh.pendB = 0;
     }
-    cluster_barrier_sync();   // every block's barriers are initialised before any remote arrival
+    // Every block's barriers are initialised before any remote arrival: all
+    // threads arrive here; only the epilogue warps, the one role that touches
+    // a peer's shared memory, wait before their first remote access (the
+    // other roles wait at teardown), so the loads start without the cluster's
+    // slowest prologue.
+    cluster_arrive_release();
     if (threadIdx.x == 0) RS_TRACE(kRtPrologue);
 
     const uint32_t tmem = sh.tmem_base;
@@ -540,6 +545,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         }
     } else {
         // --------------------------------------------------------- epilogue --
+        cluster_wait_acquire();
         const int qd = warp & 3;                     // TMEM lane quadrant of this warp
         const int row = qd * 32 + lane;              // TMEM lane = accumulator row
         const int et = threadIdx.x - 96;             // 0..127
@@ -799,6 +805,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         tmem_dealloc(tmem, kRsTmemCols);
     }
     if (threadIdx.x == 0) RS_TRACE(kRtEnd);
+    if (warp < 3) cluster_wait_acquire();   // the prologue's phase (the epilogue waited on it already)
     // no block leaves while a block of its cluster might still use its shared memory
     cluster_barrier_sync_relaxed();
 }

@@ -362,6 +362,17 @@ __device__ __forceinline__ void cluster_barrier_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
 }
+// The two halves of cluster_barrier_sync, for a thread that has work to do
+// between announcing its block's state and needing its peers': every thread
+// arrives once and waits once per phase, in that order.
+__device__ __forceinline__ void cluster_arrive_release() {
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 // the same rendezvous without memory ordering: for "nobody leaves while a block of
 // the cluster may still touch its shared memory", where every such access is
 // already accounted for by an mbarrier wait
