@@ -242,19 +242,6 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         sh.trace_once = 0u;
         sh.pendA[0] = sh.pendA[1] = sh.pendB = -1;
         fence_mbar_init();
-        const int32_t st0 = __ldcg(&a.ctl->status);
-        // acquire: the read is done before this block's count below is seen
-        const uint32_t ep0 = ld_acquire_gpu(&a.ctl->epoch);
-        if (blockIdx.x == 0) a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;   // the next launch's counter
-        sh.abort = st0 != 0;
-        sh.epoch = ep0;
-        // The last block to read the launch counter advances it for the next
-        // launch (every block of this one has read it by then; the next launch
-        // sees the new value because it starts after this one ends).
-        if (atomicAdd(&a.ctl->done, 1u) == (uint32_t)(gridDim.x - 1)) {
-            a.ctl->done = 0u;
-            a.ctl->epoch = ep0 + 1u;
-        }
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_win);
         prefetch_tmap(&tm_wout);
@@ -264,6 +251,29 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     if (warp == 2) {
         tmem_alloc(&sh.tmem_base, kRsTmemCols);
         tmem_relinquish();
+    }
+    // Launched as a programmatic dependent of the previous kernel in the stream,
+    // this block may start before that kernel has finished.  The setup above
+    // touches only this block's shared memory, TMEM and the kernel's own tensor
+    // maps; everything below reads the inputs or the workspace, which that
+    // kernel may still be writing (or, for the workspace, reading).
+    griddep_wait();
+    if (threadIdx.x == 0) {
+        griddep_launch_dependents();
+        const int32_t st0 = __ldcg(&a.ctl->status);
+        // acquire: the read is done before this block's count below is seen
+        const uint32_t ep0 = ld_acquire_gpu(&a.ctl->epoch);
+        if (blockIdx.x == 0) a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;   // the next launch's counter
+        sh.abort = st0 != 0;
+        sh.epoch = ep0;
+        // The last block to read the launch counter advances it for the next
+        // launch (every block of this one has read it by then; the next launch
+        // sees the new value because it reads it only after this one has
+        // completed: stream order, or its griddep_wait).
+        if (atomicAdd(&a.ctl->done, 1u) == (uint32_t)(gridDim.x - 1)) {
+            a.ctl->done = 0u;
+            a.ctl->epoch = ep0 + 1u;
+        }
     }
     if (warp >= 3) {
         // the chunk's union, ascending (warps 3-6 take 32-expert groups; all of a
@@ -825,13 +835,17 @@ static cudaError_t launch_decode_n(const DcArgs& a, const CUtensorMap* maps, int
     cfg.blockDim = dim3(kRsThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kRsCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // may start while the previous kernel in the stream finishes (the kernel
+    // waits for it before touching any input or the workspace)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, union_expert_decode<N>, maps[0], maps[1], maps[2], maps[3], maps[4], a);
 }
 

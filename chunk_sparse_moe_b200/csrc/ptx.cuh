@@ -46,6 +46,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Programmatic dependent launch.  griddep_wait: every grid this launch depends
+// on has completed and its memory operations are visible (returns at once for
+// a launch without a programmatic dependency).  griddep_launch_dependents: the
+// next grid in the stream may be scheduled now (it still waits in its own
+// griddep_wait until this grid has completed).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // one lane of the (converged) warp is chosen; true in that lane only
 __device__ __forceinline__ bool elect_one() {
     uint32_t p;

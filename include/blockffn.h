@@ -140,6 +140,11 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  *   fp32: any d_h, d_e >= 1.
  * Arithmetic: bf16 inputs, fp32 accumulation; the gated Swish activations are
  * rounded to bf16 between the two GEMMs; y is rounded once to dt.
+ * Ordering: stream-ordered like any kernel launch.  The single-chunk bf16 kernel
+ * (T <= n) is launched as a programmatic dependent of the preceding kernel on
+ * the stream: its blocks may start while that kernel finishes, but they set up
+ * only their own on-chip state before waiting for it to complete, so inputs
+ * produced by the preceding kernel (x, gates, weights) are read only after it.
  */
 blockffn_status blockffn_forward(const void* x, const float* gates, const void* W_r,
                                  const float* b_r, const float* gamma, float eps,

@@ -174,6 +174,36 @@ def test_deterministic_and_workspace_reuse(bffn):
     assert bffn.device_status(ws) == (0, 0)
 
 
+def test_chained_launches_read_the_previous_output(bffn):
+    """Each forward's input is the previous forward's output, launched back to back
+    on one stream with no host synchronisation: the single-chunk kernel may begin
+    before its predecessor finishes (programmatic dependent launch) and must not
+    read x, the gates or the workspace before it has.  Bit-identical to the same
+    chain with a device synchronisation after every call."""
+    w = wl.chunk32()
+    ws = bffn.Workspace.for_shapes(w.T, w.d_h, w.E, w.d_e, w.n, torch.bfloat16, False)
+    x0 = dev(w.x, torch.bfloat16)
+    W_in, W_out = dev(w.W_in, torch.bfloat16), dev(w.W_out, torch.bfloat16)
+    g = dev(w.gates, torch.float32)
+
+    def chain(sync):
+        xs = [x0]
+        for _ in range(6):
+            xs.append(bffn.forward(xs[-1], W_in, W_out, w.n, gates=g, workspace=ws))
+            if sync:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return [t.float().cpu().numpy() for t in xs[1:]]
+
+    ref = chain(True)
+    for _ in range(3):
+        got = chain(False)
+        for k, (a, b) in enumerate(zip(got, ref)):
+            assert np.array_equal(a, b), f"link {k} differs"
+    assert np.any(ref[0]) and np.all(np.isfinite(ref[-1]))
+    assert bffn.device_status(ws) == (0, 0)
+
+
 # ----------------------------------------------- the five workloads, full size --
 
 def test_workload_tiny_f32(bffn):
