@@ -157,6 +157,12 @@ __device__ __forceinline__ void cp_async_16(void* dst_smem, const void* src_glob
                  "l"(src_global)
                  : "memory");
 }
+// the same, reading src_bytes (0 or 16) and zero-filling the rest
+__device__ __forceinline__ void cp_async_16_zfill(void* dst_smem, const void* src_global, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)), "l"(src_global),
+                 "r"(src_bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
