@@ -84,17 +84,23 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 // box_rows, 2} fetches two consecutive 64-column blocks of box_rows rows and
 // lands as two [box_rows x 128 B] 128-byte-swizzled tiles, one after the other.
 // One TMA operation instead of two: the per-operation cost dominates below
-// ~32 KB.  cols must be a multiple of 128.
-bool make_map_kpair(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+// ~32 KB.  cols must be a multiple of 128.  map_kblocks is the same with nkb
+// consecutive column blocks per box (cols a multiple of 64 * nkb).
+bool map_kblocks(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                 uint32_t nkb) {
     auto fn = encode_fn();
-    if (fn == nullptr || cols % 128 != 0) return false;
+    if (fn == nullptr || cols % (64 * nkb) != 0) return false;
     cuuint64_t dims[3] = {64, rows, cols / 64};
     cuuint64_t strides[2] = {cols * 2, 128};
-    cuuint32_t box[3] = {64, box_rows, 2};
+    cuuint32_t box[3] = {64, box_rows, nkb};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_kpair(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    return map_kblocks(m, base, cols, rows, box_rows, 2);
 }
 
 // 2-D bf16 tensor [outer, inner], box {box_inner, box_outer}, no swizzle (for
@@ -178,6 +184,12 @@ blockffn_status check_shapes(int T, int d_h, int E, int d_e, int n, blockffn_dty
 }
 
 }  // namespace
+
+// for the kernels' own launchers (launch.h)
+bool bffn::make_map_kblocks(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                            uint32_t nkb) {
+    return map_kblocks(m, base, cols, rows, box_rows, nkb);
+}
 
 extern "C" {
 

@@ -10,6 +10,12 @@
 
 namespace bffn {
 
+// bf16 matrix [rows, cols] as a 3-D TMA tensor {64, row, column block}; a box
+// {64, box_rows, nkb} lands as nkb consecutive [box_rows x 128 B] 128-byte-
+// swizzled tiles (defined in abi.cu)
+bool make_map_kblocks(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                      uint32_t nkb);
+
 cudaError_t launch_route(const void* x, const void* W_r, const float* b_r, const float* gamma,
                          float eps, int T, int d_h, int E, bool bf16, float* gates,
                          cudaStream_t s);

@@ -67,6 +67,62 @@ constexpr size_t route_smem_bytes() {
            (BF16 ? sizeof(__nv_bfloat16) * (size_t)(kRtTok + 64 * EV) * kRtRaw : 0);
 }
 
+// The cluster's KS partial logit tiles [kRtTok][EP] (one per block, in shared
+// memory, complete: the caller has passed a cluster barrier) become gates: block
+// r takes tokens r*32/KS .. (r+1)*32/KS - 1, one warp per token; logit = sum over
+// ranks 0..KS-1 of their partials (+ b_r), then ReLU, the mean of squares over E
+// and the scale.
+template <int EP>
+__device__ __forceinline__ void route_finish(const float* part, int KS, int r, int t0, int Ttok, int E,
+                                             const float* __restrict__ b_r, const float* __restrict__ gamma,
+                                             float eps, float* __restrict__ gates) {
+    constexpr int NJ = EP / 32;   // experts per lane
+    const int tid = threadIdx.x;
+
+    const int tpb = kRtTok / KS;
+    const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t part_u32 = smem_u32(part);
+    for (int tt = warp; tt < tpb; tt += (int)(blockDim.x / 32)) {
+        const int tl = r * tpb + tt, gt = t0 + tl;
+        float lg[NJ];   // this lane's experts: lane + 32*j
+        float ss = 0.f;
+        // all of this lane's remote partials are requested before the first is
+        // added (the ranks' partials were written before the cluster barrier)
+        float pv[NJ][kRtMaxKS];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j)
+#pragma unroll
+            for (int q = 0; q < kRtMaxKS; ++q) {
+                pv[j][q] = 0.f;
+                if (q < KS) {
+                    const uint32_t ra = mapa_shared(part_u32 + (uint32_t)((tl * EP + lane + 32 * j) * 4), (uint32_t)q);
+                    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pv[j][q]) : "r"(ra));
+                }
+            }
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const int e = lane + 32 * j;
+            float s = 0.f;
+#pragma unroll
+            for (int q = 0; q < kRtMaxKS; ++q)
+                if (q < KS) s += pv[j][q];
+            if (b_r != nullptr && e < E) s += b_r[e];
+            const float rl = e < E ? fmaxf(s, 0.f) : 0.f;
+            lg[j] = rl;
+            ss = fmaf(rl, rl, ss);
+        }
+        ss = warp_sum(ss);
+        const float denom = sqrtf(ss / (float)E + eps);
+        if (gt < Ttok) {
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                const int e = lane + 32 * j;
+                if (e < E) gates[(size_t)gt * E + e] = lg[j] > 0.f ? gamma[e] * lg[j] / denom : 0.f;
+            }
+        }
+    }
+}
+
 template <typename T, int EV>
 __global__ void __launch_bounds__(kRtThreads) route_kernel(
     const T* __restrict__ x, const T* __restrict__ W_r, const float* __restrict__ b_r,
@@ -160,52 +216,159 @@ __global__ void __launch_bounds__(kRtThreads) route_kernel(
             *reinterpret_cast<float4*>(part + (2 * tx + i) * EP + 64 * v + 4 * ty) =
                 make_float4(acc[i][4 * v], acc[i][4 * v + 1], acc[i][4 * v + 2], acc[i][4 * v + 3]);
     cluster_barrier_sync();   // every block's partials are written
+    route_finish<EP>(part, KS, r, t0, Ttok, E, b_r, gamma, eps, gates);
+    cluster_barrier_sync();   // no block leaves while a peer may still read its partials
+}
 
-    // block r finishes tokens r*TPB .. r*TPB + TPB - 1 of the cluster's 32, one warp
-    // per token: logit = sum over ranks 0..KS-1 of their partials (+ b_r)
-    const int tpb = kRtTok / KS;
-    const int warp = tid >> 5, lane = tid & 31;
-    const uint32_t part_u32 = smem_u32(part);
-    for (int tt = warp; tt < tpb; tt += kRtThreads / 32) {
-        const int tl = r * tpb + tt, gt = t0 + tl;
-        float lg[EV * 2];   // this lane's experts: lane + 32*j
-        float ss = 0.f;
-        // all of this lane's remote partials are requested before the first is
-        // added (the ranks' partials were written before the cluster barrier)
-        float pv[2 * EV][kRtMaxKS];
+// ---------------------------------------------------------------------------
+// bf16 with d_h % 256 == 0: the same cluster split, the products on the tensor
+// cores.  A block's slice of d_h goes through in groups of 256 k: one TMA box
+// per 128-expert tile of W_r ({64, 128, 4}: 64 KB) and one for x ({64, 32, 4}:
+// 16 KB), each landing as four 128-byte-swizzled k-blocks; then 16 MMAs per
+// expert tile (experts as M = 128, the 32 tokens as N, K = 16), accumulating in
+// TMEM.  Experts past E and tokens past T are zeros from the boxes' out-of-range
+// fill.  The accumulators come back with tcgen05.ld into the partial tile, and
+// route_finish adds the ranks' tiles as in the CUDA-core kernel.  Every wait is
+// bounded; a block that runs out writes NaN partials, so the gates it feeds
+// come out NaN rather than wrong-but-plausible.
+constexpr int kRqThreads = 128;
+constexpr int kRqKg = 256;                   // k per group
+constexpr uint64_t kRqWaitNs = 2000000000ull;
+
+template <int ET>
+constexpr size_t route_tc_smem_bytes() {
+    return 1024 + (size_t)ET * 65536 + 16384 + sizeof(float) * kRtTok * 128 * ET;
+}
+
+__device__ __forceinline__ bool rq_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > kRqWaitNs) return false;
+    return true;
+}
+
+template <int ET>
+__global__ void __launch_bounds__(kRqThreads, 1) route_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+    const float* __restrict__ b_r, const float* __restrict__ gamma, float eps, int Ttok, int E, int KS,
+    int slice, float* __restrict__ gates) {
+    constexpr int EP = 128 * ET;
+    constexpr uint32_t kCols = 32 * ET;   // one 32-column accumulator per expert tile (a power of 2)
+    extern __shared__ uint8_t rq_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rq_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* wsm = sm;                                   // [ET][4 k-blocks][128 rows x 128 B]
+    uint8_t* xsm = sm + ET * 65536;                      // [4 k-blocks][32 rows x 128 B]
+    float* part = reinterpret_cast<float*>(xsm + 16384);  // [kRtTok][EP]
+    __shared__ __align__(8) uint64_t full, mma_bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ int ok_s;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kRtTok;
+    const int r = (int)cluster_ctarank();
+    if (threadIdx.x == 0) {
+        mbar_init(&full, 1);
+        mbar_init(&mma_bar, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_w);
+        ok_s = 1;
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_base, kCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    griddep_launch_dependents();
+    const uint32_t tmem = tmem_base;
+    if (threadIdx.x == 0) {
+        const uint32_t idesc = idesc_bf16_f32(128, kRtTok);
+        const uint64_t pol = policy_evict_last();
+        const uint64_t dw = sw128_kmajor_desc(smem_u32(wsm)), dx = sw128_kmajor_desc(smem_u32(xsm));
+        bool ok = true;
+        const int ng = slice / kRqKg;
+        for (int g = 0; g < ng && ok; ++g) {
+            const int kb0 = (r * slice + g * kRqKg) / 64;
+            mbar_arrive_expect_tx(&full, (uint32_t)(ET * 65536 + 16384));
 #pragma unroll
-        for (int j = 0; j < 2 * EV; ++j)
+            for (int et = 0; et < ET; ++et) tma_load_3d(wsm + et * 65536, &tm_w, &full, 0, et * 128, kb0, pol);
+            tma_load_3d(xsm, &tm_x, &full, 0, t0, kb0, pol);
+            ok = rq_wait(&full, (uint32_t)(g & 1));
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < kRtMaxKS; ++q) {
-                pv[j][q] = 0.f;
-                if (q < KS) {
-                    const uint32_t ra = mapa_shared(part_u32 + (uint32_t)((tl * EP + lane + 32 * j) * 4), (uint32_t)q);
-                    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pv[j][q]) : "r"(ra));
-                }
-            }
+            for (int et = 0; et < ET; ++et)
 #pragma unroll
-        for (int j = 0; j < 2 * EV; ++j) {
-            const int e = lane + 32 * j;
-            float s = 0.f;
+                for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
-            for (int q = 0; q < kRtMaxKS; ++q)
-                if (q < KS) s += pv[j][q];
-            if (b_r != nullptr && e < E) s += b_r[e];
-            const float rl = e < E ? fmaxf(s, 0.f) : 0.f;
-            lg[j] = rl;
-            ss = fmaf(rl, rl, ss);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(tmem + (uint32_t)(32 * et),
+                                  dw + (uint64_t)((et * 65536 + kb * 16384 + kk * 32) >> 4),
+                                  dx + (uint64_t)((kb * 4096 + kk * 32) >> 4), idesc,
+                                  (g > 0 || kb > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&mma_bar);
+            // the buffers are reloaded (next group) or the accumulators read only
+            // once these MMAs are done
+            ok = rq_wait(&mma_bar, (uint32_t)(g & 1));
         }
-        ss = warp_sum(ss);
-        const float denom = sqrtf(ss / (float)E + eps);
-        if (gt < Ttok) {
-#pragma unroll
-            for (int j = 0; j < 2 * EV; ++j) {
-                const int e = lane + 32 * j;
-                if (e < E) gates[(size_t)gt * E + e] = lg[j] > 0.f ? gamma[e] * lg[j] / denom : 0.f;
-            }
+        if (!ok) {
+            ok_s = 0;
+            // give copies still in flight a bounded chance to land before leaving
+            rq_wait(&full, 0u);
+            rq_wait(&full, 1u);
         }
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const bool ok = ok_s != 0;
+    // accumulator row = TMEM lane = expert (warp w holds experts 32w .. 32w+31 of each tile)
+#pragma unroll
+    for (int et = 0; et < ET; ++et) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * et), v);
+        tmem_ld_wait();
+        const int e = 128 * et + 32 * warp + lane;
+#pragma unroll
+        for (int t = 0; t < kRtTok; ++t) part[t * EP + e] = ok ? __uint_as_float(v[t]) : __int_as_float(0x7fc00000);
+    }
+    tc_fence_before();
+    cluster_barrier_sync();   // every block's partials are written
+    route_finish<EP>(part, KS, r, t0, Ttok, E, b_r, gamma, eps, gates);
     cluster_barrier_sync();   // no block leaves while a peer may still read its partials
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kCols);
+    }
+}
+
+template <int ET>
+static cudaError_t launch_route_tc(const __nv_bfloat16* x, const __nv_bfloat16* W_r, const float* b_r,
+                                   const float* gamma, float eps, int Ttok, int d_h, int E, int KS, float* gates,
+                                   cudaStream_t s) {
+    CUtensorMap mx, mw;
+    if (!make_map_kblocks(&mx, x, (uint64_t)d_h, (uint64_t)Ttok, kRtTok, 4) ||
+        !make_map_kblocks(&mw, W_r, (uint64_t)d_h, (uint64_t)E, 128, 4))
+        return cudaErrorInvalidValue;
+    const size_t smem = route_tc_smem_bytes<ET>();
+    cudaError_t err =
+        cudaFuncSetAttribute(route_tc_kernel<ET>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((Ttok + kRtTok - 1) / kRtTok, KS, 1);
+    cfg.blockDim = dim3(kRqThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = KS;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, route_tc_kernel<ET>, mx, mw, b_r, gamma, eps, Ttok, E, KS, d_h / KS, gates);
 }
 
 template <typename T, int EV>
@@ -247,6 +410,15 @@ cudaError_t launch_route(const void* x, const void* W_r, const float* b_r, const
                          float eps, int T, int d_h, int E, bool bf16, float* gates,
                          cudaStream_t s) {
     if (T == 0) return cudaSuccess;
+    if (bf16 && d_h % kRqKg == 0 && E <= 256) {
+        // tensor cores: KS slices of whole 256-k groups
+        int KS = kRtMaxKS;
+        while (KS > 1 && d_h % (kRqKg * KS) != 0) KS /= 2;
+        const auto* xb = static_cast<const __nv_bfloat16*>(x);
+        const auto* wb = static_cast<const __nv_bfloat16*>(W_r);
+        return E <= 128 ? launch_route_tc<1>(xb, wb, b_r, gamma, eps, T, d_h, E, KS, gates, s)
+                        : launch_route_tc<2>(xb, wb, b_r, gamma, eps, T, d_h, E, KS, gates, s);
+    }
     if (bf16)
         return launch_route_t(static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W_r), b_r,
                               gamma, eps, T, d_h, E, gates, s);

@@ -89,6 +89,17 @@ def test_route_seq4096_bf16(bffn):
     _check_route(bffn, wl.seq4096())
 
 
+@pytest.mark.parametrize("T,d_h,E,bias", [
+    (45, 512, 192, -0.8),    # two 128-expert tiles, d_h in 2 slices, ragged last token tile
+    (7, 4096, 256, None),    # fewer tokens than a tile, two 256-wide k-groups per slice
+    (70, 2304, 64, -0.5),    # d_h 9 x 256: one slice of nine k-groups
+    (33, 320, 48, None),     # d_h not a multiple of 256: the CUDA-core router
+])
+def test_route_bf16_shapes(bffn, T, d_h, E, bias):
+    w = wl.make_routed("route_shape", T, 32, d_h, E, 1, "bf16", seed=T + E, bias_shift=bias)
+    _check_route(bffn, w)
+
+
 def test_route_edge_rows(bffn):
     """A row whose logits are all <= 0 gives zero gates; negative gamma keeps the sign."""
     w = wl.make_routed("edge", 40, 8, 128, 16, 128, "bf16", seed=3, bias_shift=-0.8)
