@@ -381,48 +381,69 @@ union_expert_forward_tc(const __grid_constant__ CUtensorMap tm_x,
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer --
-        if (lane == 0) {
+        // The whole warp runs the loop with warp-wide waits and one elected lane
+        // issues: a loop run by one lane while the other 31 wait issued tcgen05
+        // work at about half the rate.  Each operand descriptor is the stage's
+        // base descriptor plus a constant, and the next stage's barriers are
+        // tested while the current stage's MMAs issue.
+        {
+            const bool leader = elect_one();
             const uint32_t idesc = idesc_bf16_f32(128, N);
+            const uint64_t desc0 = sw128_kmajor_desc(smem_u32(smem));
             SegIter it;
             it.init(aLo, aHi, bLo, bHi);
             Seg sg;
             long long i = 0;
+            int st = 0;
+            uint32_t ph = 0u;
+            uint32_t rw = 0u, rh = 0u;   // the current stage's barriers as last tested
             uint32_t acc_i = 0;
-            bool stop = sh.abort != 0;
+            bool stop = __shfl_sync(0xffffffffu, sh.abort, 0) != 0;
             while (!stop && it.next(a, tb, sg)) {
                 const int ab = (int)(acc_i % kNAcc);
                 const uint32_t aph = (acc_i / kNAcc) & 1u;
-                if (!wait_bar(&sh.acc_empty[ab], aph ^ 1u, limit, &sh.abort, a.ctl, kWaitAccEmpty))
+                if (!wait_bar_warp(&sh.acc_empty[ab], aph ^ 1u, limit, &sh.abort, a.ctl, kWaitAccEmpty))
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(ab * 32);
                 for (long long j = sg.lo; j < sg.hi; ++j, ++i) {
-                    const int st = (int)(i % kStages);
-                    const uint32_t ph = (uint32_t)((i / kStages) & 1);
-                    if (!wait_bar(&sh.full_w[st], ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
-                        !wait_bar(&sh.full_h[st], ph, limit, &sh.abort, a.ctl, kWaitFullH)) {
+                    if (!__all_sync(0xffffffffu, rw & rh) &&
+                        (!wait_bar_warp(&sh.full_w[st], ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
+                         !wait_bar_warp(&sh.full_h[st], ph, limit, &sh.abort, a.ctl, kWaitFullH))) {
                         stop = true;
                         break;
                     }
                     tc_fence_after();
-                    fence_proxy_async_smem();   // activation tiles were written by cp.async
-                    if (i == 0) BFFN_TRACE(kTrFirstFull);
-                    if (sg.kind == 1) BFFN_TRACE_ONCE(kTrFirstBMma);
-                    const uint32_t wb = smem_u32(smem + st * kStageBytes);
-                    const uint32_t xb = wb + kWBytes;
+                    const int st_n = st + 1 == kStages ? 0 : st + 1;
+                    const uint32_t ph_n = st + 1 == kStages ? ph ^ 1u : ph;
+                    rw = mbar_test_wait(&sh.full_w[st_n], ph_n);
+                    rh = mbar_test_wait(&sh.full_h[st_n], ph_n);
+                    if (leader) {
+                        fence_proxy_async_smem();   // activation tiles were written by cp.async
+                        if (i == 0) BFFN_TRACE(kTrFirstFull);
+                        if (sg.kind == 1) BFFN_TRACE_ONCE(kTrFirstBMma);
+                        const uint64_t ds = desc0 + (uint64_t)(st * (kStageBytes >> 4));
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(d, sw128_kmajor_desc(wb + kk * 32), sw128_kmajor_desc(xb + kk * 32),
-                                  idesc, (j > sg.lo || kk > 0) ? 1u : 0u);
-                    umma_commit(&sh.empty[st]);
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d, ds + (uint64_t)((kk * 32) >> 4), ds + (uint64_t)((kWBytes + kk * 32) >> 4),
+                                      idesc, (j > sg.lo || kk > 0) ? 1u : 0u);
+                        umma_commit(&sh.empty[st]);
+                    }
+                    __syncwarp();
+                    st = st_n;
+                    ph = ph_n;
                 }
                 if (stop) break;
-                umma_commit(&sh.acc_full[ab]);
-                if (sg.kind == 0) BFFN_TRACE(kTrLastACommit);
-                BFFN_TRACE(kTrLastCommit);
+                if (leader) {
+                    umma_commit(&sh.acc_full[ab]);
+                    if (sg.kind == 0) BFFN_TRACE(kTrLastACommit);
+                    BFFN_TRACE(kTrLastCommit);
+                }
+                __syncwarp();
                 ++acc_i;
             }
-            umma_commit(&sh.mma_done);
+            if (leader) umma_commit(&sh.mma_done);
+            __syncwarp();
         }
     } else if (warp == 2) {
         // ------------------------------------- gated-activation loader --
