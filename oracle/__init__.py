@@ -14,6 +14,7 @@ passages they follow:
 * ``forward_dense``       -- y = sum over ALL experts of gate * expert(x)
 * ``forward_chunk_union`` -- union experts over whole chunks, masked after compute
 * ``sparsity``            -- token-level and L-token chunk-level sparsity
+* ``residual_layernorm``  -- LayerNorm(y + x) over the hidden dimension
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against facts that do
 not come from this code (closed forms, a library MLP, brute force, invariants).
@@ -67,6 +68,8 @@ def _load():
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, _D]
         lib.oracle_sparsity.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int, _D]
+        lib.oracle_residual_layernorm.argtypes = [_D, _D, _D, _D, ctypes.c_double, ctypes.c_int,
+                                                  ctypes.c_int, _D]
         _lib = lib
     return _lib
 
@@ -149,3 +152,15 @@ def sparsity(gates, L: int):
     out = np.empty(2, np.float64)
     lib.oracle_sparsity(_p(g, _D), T, E, int(L), _p(out, _D))
     return float(out[0]), float(out[1])
+
+
+def residual_layernorm(y, x, ln_gamma, ln_beta, eps: float) -> np.ndarray:
+    """out = LayerNorm(y + x) over the hidden dimension (scale ln_gamma, shift ln_beta), fp64."""
+    lib = _load()
+    y, x, g, b = _f64(y), _f64(x), _f64(ln_gamma), _f64(ln_beta)
+    T, d_h = x.shape
+    assert y.shape == (T, d_h) and g.shape == (d_h,) and b.shape == (d_h,)
+    out = np.empty((T, d_h), np.float64)
+    lib.oracle_residual_layernorm(_p(y, _D), _p(x, _D), _p(g, _D), _p(b, _D), float(eps), T, d_h,
+                                  _p(out, _D))
+    return out

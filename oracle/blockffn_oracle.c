@@ -249,3 +249,39 @@ void oracle_sparsity(const double* gates, int T, int E, int L, double* out)
     out[0] = (double)zero / ((double)T * E);
     out[1] = (double)inactive / ((double)C * E);
 }
+
+/*
+ * Residual and LayerNorm after the layer.  [SKILL] "Full BlockFFN Layer with
+ * Combined Losses": the layer's output is its expert sum plus its input, put
+ * through a LayerNorm over the hidden dimension (nn.LayerNorm(hidden_dim): a
+ * learnable per-feature scale and shift, population variance).
+ *
+ *   v[t,k]   = y[t,k] + x[t,k]
+ *   mu[t]    = (1/d_h) sum_k v[t,k]
+ *   var[t]   = (1/d_h) sum_k (v[t,k] - mu[t])^2
+ *   out[t,k] = ln_gamma[k] * (v[t,k] - mu[t]) / sqrt(var[t] + eps) + ln_beta[k]
+ *
+ * Reading: eps is an argument (nn.LayerNorm's default is 1e-5); the variance is
+ * taken around the mean in a second pass.
+ */
+void oracle_residual_layernorm(const double* y, const double* x, const double* ln_gamma,
+                               const double* ln_beta, double eps, int T, int d_h, double* out)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const double* yr = y + (size_t)t * d_h;
+        const double* xr = x + (size_t)t * d_h;
+        double* o = out + (size_t)t * d_h;
+        double mu = 0.0;
+        for (int k = 0; k < d_h; ++k) mu += yr[k] + xr[k];
+        mu /= (double)d_h;
+        double var = 0.0;
+        for (int k = 0; k < d_h; ++k) {
+            const double dv = (yr[k] + xr[k]) - mu;
+            var += dv * dv;
+        }
+        var /= (double)d_h;
+        const double rstd = 1.0 / sqrt(var + eps);
+        for (int k = 0; k < d_h; ++k) o[k] = ln_gamma[k] * ((yr[k] + xr[k]) - mu) * rstd + ln_beta[k];
+    }
+}

@@ -11,11 +11,14 @@ from a fact the pages or mathematics fix:
 * pure-Python brute force on tiny shapes, and an exhaustive enumeration of
   every mask of a tiny chunk for the union lists;
 * the router equals torch's own ``rms_norm`` of ``relu(W_r x + b)``;
-* hand-derived worked examples (tests/golden/hand_examples.json).
+* hand-derived worked examples (tests/golden/hand_examples.json);
+* the residual LayerNorm equals torch's ``layer_norm`` of y + x, and its closed
+  forms (constant row -> shift, unit moments, scale invariance).
 
 ``test_pins_catch_planted_mistakes`` compiles mutated copies of the oracle
 (a dropped expert, a sign flip in Swish, a transposed weight index, the wrong
-token's gate, a wrong RMS mean, a shifted token bit, a scrambled union list)
+token's gate, a wrong RMS mean, a shifted token bit, a scrambled union list, a
+LayerNorm without the residual, a sample variance)
 and checks that at least one pin fails for each.
 """
 from __future__ import annotations
@@ -265,6 +268,45 @@ def pin_sparsity(orc) -> float:
     return worst
 
 
+def pin_residual_layernorm_torch(orc) -> float:
+    """LayerNorm(y + x) equals torch's own layer_norm of the sum (fp64, a library
+    routine), for a ragged width, random scale/shift and two eps values."""
+    import torch
+    worst = 0.0
+    for seed, (T, d_h, eps) in enumerate([(5, 300, 1e-5), (3, 64, 0.25), (1, 7, 1e-5)]):
+        rng = np.random.default_rng(300 + seed)
+        y, x = rng.standard_normal((T, d_h)) * 3.0, rng.standard_normal((T, d_h))
+        g, b = rng.uniform(-2.0, 2.0, d_h), rng.standard_normal(d_h)
+        ref = torch.nn.functional.layer_norm(torch.from_numpy(y + x), (d_h,), torch.from_numpy(g),
+                                             torch.from_numpy(b), eps).numpy()
+        worst = max(worst, _rel(orc.residual_layernorm(y, x, g, b, eps), ref))
+    return worst
+
+
+def pin_residual_layernorm_closed_forms(orc) -> float:
+    """Closed forms: a constant row gives exactly the shift; with unit scale and
+    zero shift a row has mean 0 and mean square var / (var + eps); scaling y + x
+    by a > 0 (eps = 0) leaves the output unchanged."""
+    rng = np.random.default_rng(11)
+    d_h = 96
+    worst = 0.0
+    b = rng.standard_normal(d_h)
+    c = np.full((2, d_h), 0.75)
+    out = orc.residual_layernorm(c, -0.25 * np.ones((2, d_h)), rng.uniform(0.5, 2, d_h), b, 1e-5)
+    worst = max(worst, float(np.max(np.abs(out - b))))
+    y, x = rng.standard_normal((4, d_h)), rng.standard_normal((4, d_h))
+    eps = 0.1
+    out = orc.residual_layernorm(y, x, np.ones(d_h), np.zeros(d_h), eps)
+    v = y + x
+    var = np.mean((v - v.mean(1, keepdims=True)) ** 2, axis=1)
+    worst = max(worst, float(np.max(np.abs(out.mean(1)))))
+    worst = max(worst, float(np.max(np.abs((out ** 2).mean(1) - var / (var + eps)))))
+    o1 = orc.residual_layernorm(y, x, np.ones(d_h), np.zeros(d_h), 0.0)
+    o2 = orc.residual_layernorm(3.5 * y, 3.5 * x, np.ones(d_h), np.zeros(d_h), 0.0)
+    worst = max(worst, _rel(o2, o1))
+    return worst
+
+
 PINS = {
     "all_on_dense_mlp": (pin_all_on_dense_mlp, 1e-12),
     "one_active_expert": (pin_one_active_expert, 1e-12),
@@ -275,6 +317,8 @@ PINS = {
     "rms_identity": (pin_rms_identity, 1e-13),
     "hand_examples": (pin_hand_examples, 1e-15),
     "sparsity": (pin_sparsity, 0.0),
+    "residual_layernorm_torch": (pin_residual_layernorm_torch, 1e-13),
+    "residual_layernorm_closed_forms": (pin_residual_layernorm_closed_forms, 1e-12),
 }
 
 
@@ -320,6 +364,11 @@ MUTANTS = {
     # union ignores the ragged tail guard
     "wrong_idx_order": ("if (bits != 0u) idx[(size_t)c * E + cnt++] = e;",
                         "if (bits != 0u) idx[(size_t)c * E + cnt++] = E - 1 - e;"),
+    # the residual dropped from the LayerNorm's input
+    "ln_no_residual": ("for (int k = 0; k < d_h; ++k) mu += yr[k] + xr[k];",
+                       "for (int k = 0; k < d_h; ++k) mu += yr[k];"),
+    # the sample (n - 1) variance instead of nn.LayerNorm's population variance
+    "ln_sample_variance": ("var /= (double)d_h;", "var /= (double)(d_h - 1);"),
 }
 
 
