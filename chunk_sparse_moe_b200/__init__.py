@@ -7,8 +7,8 @@ library's kernels; PyTorch only provides device memory and streams.
 """
 from .api import (BlockFFNError, Workspace, chunk_union, debug_set_trace, debug_skip_flag, device_status,
                   forward,
-                  num_sms, route, set_wait_limit_ns, version, workspace_bytes)
+                  num_sms, residual_layernorm, route, set_wait_limit_ns, version, workspace_bytes)
 
-__all__ = ["BlockFFNError", "Workspace", "chunk_union", "debug_set_trace", "debug_skip_flag",
+__all__ = ["BlockFFNError", "Workspace", "chunk_union", "debug_set_trace", "debug_skip_flag", "residual_layernorm",
            "device_status",
            "forward", "num_sms", "route", "set_wait_limit_ns", "version", "workspace_bytes"]

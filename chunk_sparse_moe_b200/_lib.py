@@ -32,6 +32,8 @@ SIGNATURES = {
                                c_int, c_int, c_void_p, c_void_p]),
     "blockffn_chunk_union": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                      c_void_p, c_void_p]),
+    "blockffn_residual_layernorm": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_int,
+                                            c_int, c_int, c_void_p, c_void_p]),
     "blockffn_forward_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int,
                                                     c_int]),
     "blockffn_workspace_reset": (c_int, [c_void_p, c_size_t, c_void_p]),

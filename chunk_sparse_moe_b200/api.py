@@ -86,6 +86,19 @@ def route(x: torch.Tensor, W_r: torch.Tensor, gamma: torch.Tensor, eps: float,
     return out
 
 
+def residual_layernorm(y: torch.Tensor, x: torch.Tensor, ln_gamma: torch.Tensor,
+                       ln_beta: torch.Tensor, eps: float = 1e-5,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out [T, d_h] = LayerNorm(y + x) over d_h (scale ln_gamma, shift ln_beta, fp32)."""
+    T, d_h = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib.blockffn_residual_layernorm(_ptr(y), _ptr(x), _ptr(ln_gamma), _ptr(ln_beta), float(eps),
+                                         T, d_h, _dtype_code(x), _ptr(out), _stream())
+    _check(st, "blockffn_residual_layernorm")
+    return out
+
+
 def chunk_union(gates: torch.Tensor, n: int):
     """Per-chunk union of active experts: (counts [C], idx [C,E], tmask [C,E] as int32)."""
     T, E = gates.shape

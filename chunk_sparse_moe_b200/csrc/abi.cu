@@ -236,6 +236,19 @@ blockffn_status blockffn_route(const void* x, const void* W_r, const float* b_r,
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "route launch");
 }
 
+blockffn_status blockffn_residual_layernorm(const void* y, const void* x, const float* ln_gamma,
+                                           const float* ln_beta, float eps, int T, int d_h, blockffn_dtype dt,
+                                           void* out, void* stream) {
+    if (dt != BLOCKFFN_F32 && dt != BLOCKFFN_BF16) return fail(BLOCKFFN_ERR_INVALID_ARG, "unknown dtype");
+    if (T < 0 || d_h < 1) return fail(BLOCKFFN_ERR_INVALID_ARG, "bad shape (T = %d, d_h = %d)", T, d_h);
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(BLOCKFFN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    if (T == 0) return BLOCKFFN_OK;
+    if (!y || !x || !ln_gamma || !ln_beta || !out) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
+    cudaError_t e = launch_residual_layernorm(y, x, ln_gamma, ln_beta, eps, T, d_h, dt == BLOCKFFN_BF16, out,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "residual layernorm launch");
+}
+
 blockffn_status blockffn_chunk_union(const float* gates, int T, int E, int n, int32_t* counts,
                                      int32_t* idx, uint32_t* tmask, void* stream) {
     if (T < 0 || E < 1 || E > 256 || n < 1 || n > 32) return fail(BLOCKFFN_ERR_INVALID_ARG, "bad shape");

@@ -20,6 +20,9 @@ cudaError_t launch_route(const void* x, const void* W_r, const float* b_r, const
                          float eps, int T, int d_h, int E, bool bf16, float* gates,
                          cudaStream_t s);
 
+cudaError_t launch_residual_layernorm(const void* y, const void* x, const float* ln_gamma, const float* ln_beta,
+                                      float eps, int T, int d_h, bool bf16, void* out, cudaStream_t s);
+
 cudaError_t launch_chunk_union(const float* gates, int T, int E, int n, int32_t* counts,
                                int32_t* idx, uint32_t* tmask, cudaStream_t s);
 

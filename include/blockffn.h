@@ -106,6 +106,24 @@ blockffn_status blockffn_chunk_union(const float* gates, int T, int E, int n,
                                      void* stream);
 
 /*
+ * blockffn_residual_layernorm -- the layer's closing step, out = LayerNorm(y + x)
+ * over the hidden dimension:
+ *   v = y + x;  mu = mean_k v;  var = mean_k (v - mu)^2  (population variance);
+ *   out[t,k] = ln_gamma[k] * (v[t,k] - mu) / sqrt(var + eps) + ln_beta[k].
+ * Pages: "BlockFFN: Sparse Mixture-of-Experts Optimized for End-Device Deployment",
+ * Full BlockFFN Layer with Combined Losses (the expert sum plus the input, through
+ * nn.LayerNorm(hidden_dim); its default eps is 1e-5).
+ * y, x, out [T, d_h] in dtype dt (out may alias y or x: every element is read
+ * before it is written); ln_gamma, ln_beta [d_h] fp32; eps finite and >= 0.
+ * Arithmetic: fp32 from the dt inputs, the sums in a fixed order, out rounded once
+ * to dt.  Stream-ordered; launched as a programmatic dependent of the preceding
+ * kernel (it reads nothing before that kernel has completed).
+ */
+blockffn_status blockffn_residual_layernorm(const void* y, const void* x, const float* ln_gamma,
+                                           const float* ln_beta, float eps, int T, int d_h,
+                                           blockffn_dtype dt, void* out, void* stream);
+
+/*
  * blockffn_forward_workspace_bytes -- size of the scratch buffer blockffn_forward
  * needs for these shapes (0 when the shapes are invalid).  with_router != 0 when
  * the gates will come from the router (the workspace then also holds them).

@@ -215,6 +215,60 @@ def test_chained_launches_read_the_previous_output(bffn):
     assert bffn.device_status(ws) == (0, 0)
 
 
+# ------------------------------------------------- residual + LayerNorm --
+
+def test_residual_layernorm_after_the_decode_step(bffn):
+    """out = LayerNorm(y + x) on the decode step's own output: against the oracle
+    given the GPU's y (the step alone) and given the oracle's y (the layer)."""
+    w = wl.chunk32()
+    y, g = run_gpu(w)
+    rng = np.random.default_rng(8)
+    lg = rng.uniform(0.5, 1.5, w.d_h).astype(np.float32)
+    lb = (0.1 * rng.standard_normal(w.d_h)).astype(np.float32)
+    x = dev(w.x, torch.bfloat16)
+    out = to_np64(bffn.residual_layernorm(dev(y, torch.bfloat16), x, dev(lg, torch.float32),
+                                          dev(lb, torch.float32), 1e-5))
+    assert_close(out, oracle.residual_layernorm(y, w.x, lg, lb, 1e-5), "bf16", "layernorm step")
+    y_ref = oracle.forward_dense(w.x, g, w.W_in, w.W_out)
+    assert_close(out, oracle.residual_layernorm(y_ref, w.x, lg, lb, 1e-5), "bf16", "layer")
+
+
+@pytest.mark.parametrize("T,d_h,dt", [(5, 300, "f32"), (1, 7, "f32"), (33, 2048, "bf16"), (3, 4096, "bf16")])
+def test_residual_layernorm_shapes(bffn, T, d_h, dt):
+    rng = np.random.default_rng(T * 7 + d_h)
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    y = wl.bf16_round(3.0 * rng.standard_normal((T, d_h))) if dt == "bf16" else rng.standard_normal((T, d_h))
+    x = wl.bf16_round(rng.standard_normal((T, d_h))) if dt == "bf16" else rng.standard_normal((T, d_h))
+    lg = rng.uniform(-2.0, 2.0, d_h).astype(np.float32)
+    lb = rng.standard_normal(d_h).astype(np.float32)
+    out = to_np64(bffn.residual_layernorm(dev(y, tdt), dev(x, tdt), dev(lg, torch.float32),
+                                          dev(lb, torch.float32), 1e-5))
+    assert_close(out, oracle.residual_layernorm(y, x, lg, lb, 1e-5), dt, f"layernorm {T}x{d_h}")
+
+
+def test_residual_layernorm_in_place_and_edge_rows(bffn):
+    """Writing over y gives the same bits; a row whose y + x is constant gives the
+    shift exactly; no rows is a no-op."""
+    rng = np.random.default_rng(21)
+    T, d_h = 4, 2048
+    y = dev(wl.bf16_round(rng.standard_normal((T, d_h))), torch.bfloat16)
+    x = dev(wl.bf16_round(rng.standard_normal((T, d_h))), torch.bfloat16)
+    lg = dev(rng.uniform(0.5, 2.0, d_h).astype(np.float32), torch.float32)
+    lb_np = wl.bf16_round(rng.standard_normal(d_h)).astype(np.float32)
+    lb = dev(lb_np, torch.float32)
+    ref = bffn.residual_layernorm(y, x, lg, lb, 1e-5).clone()
+    y2 = y.clone()
+    bffn.residual_layernorm(y2, x, lg, lb, 1e-5, out=y2)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, ref)
+    yc = torch.full((2, d_h), 0.75, dtype=torch.bfloat16, device="cuda")
+    xc = torch.full((2, d_h), -0.25, dtype=torch.bfloat16, device="cuda")
+    oc = bffn.residual_layernorm(yc, xc, lg, lb, 1e-5)
+    assert np.array_equal(to_np64(oc), np.broadcast_to(lb_np.astype(np.float64), (2, d_h)))
+    e = torch.empty((0, d_h), dtype=torch.bfloat16, device="cuda")
+    assert bffn.residual_layernorm(e, e, lg, lb, 1e-5).shape == (0, d_h)
+
+
 # ----------------------------------------------- the five workloads, full size --
 
 def test_workload_tiny_f32(bffn):
