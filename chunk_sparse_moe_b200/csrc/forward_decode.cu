@@ -33,10 +33,19 @@
 // block of rank q, which adds the 4 contributions in rank order (a fixed order)
 // and writes those 32 rows of y.
 //
-// Roles (224 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM owner
-// and h' loader, warps 3-6 epilogue.  Every wait is bounded; a timeout records
-// BLOCKFFN_ERR_TIMEOUT and the block winds down without leaving copies in
-// flight.
+// Roles (224 threads): warp 0 TMA producer (one lane), warp 1 MMA issuer (the
+// whole warp runs its loops and waits, one elected lane issues), warp 2 TMEM
+// owner and h' loader, warps 3-6 epilogue.  Every wait is bounded; a timeout
+// records BLOCKFFN_ERR_TIMEOUT and the block winds down without leaving copies
+// in flight.
+//
+// Launch.  A programmatic dependent of the previous kernel on the stream: a
+// block initialises its barriers, allocates TMEM and prefetches its tensor maps,
+// then waits for that kernel (griddepcontrol.wait) before it reads any input or
+// the workspace.  The cluster barrier after set-up is split: every thread
+// arrives, but only the epilogue warps, the one role that writes into a peer's
+// shared memory, wait before their first remote access; the other roles wait
+// at teardown.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
