@@ -27,7 +27,8 @@
 // finishes the pair's A unit sets after writing the gated activations.
 //
 // Roles (224 threads): warp 0 issues the weight/x TMA loads, warp 1 issues the
-// MMAs (one thread), warp 2 owns TMEM and copies gated activations into the
+// MMAs (the whole warp runs the loop, one elected lane issues), warp 2 owns
+// TMEM and copies gated activations into the
 // stages once their flag is set, warps 3-6 drain the accumulators (TMEM ->
 // registers) and do the split reductions, Swish, gate, mask and stores.
 #include <cuda.h>
