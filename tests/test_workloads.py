@@ -101,3 +101,17 @@ def test_seq4096_router_sparsity():
     assert abs(tls - (1 - p_on)) < 0.03
     # neighbouring tokens share experts: CLS is far above the i.i.d. value
     assert cls8 > (1 - p_on) ** 8 + 0.2
+
+
+def test_accept_lengths_match_their_closed_form():
+    """The synthetic verification outcomes: 1 .. n + 1 tokens per step, mean
+    1 + sum_k p^k (accepted prefix of a geometric run plus the verifier's own
+    token)."""
+    for n, p in [(32, 0.8), (8, 0.5), (32, 0.0)]:
+        a = wl.accept_lengths(3, 100_000, n, p)
+        assert a.min() >= 1 and a.max() <= n + 1
+        m = wl.accept_mean(n, p)
+        sd = max(float(a.std()), 1e-12)
+        assert abs(a.mean() - m) <= 4.0 * sd / np.sqrt(a.size) + 1e-12, (n, p, a.mean(), m)
+    assert np.all(wl.accept_lengths(0, 10, 32, 0.0) == 1)
+    assert np.all(wl.accept_lengths(0, 10, 32, 1.0) == 33)

@@ -233,3 +233,35 @@ def markov_closed_forms(a: float, b: float, L: int) -> dict:
     """
     p_off = b / (a + b)
     return {"tls": p_off, "cls": p_off * (1.0 - a) ** (L - 1)}
+
+
+def layer_stack(L: int, n: int, d_h: int, E: int, d_e: int, dtype: str, regime: str = "markov80",
+                seed: int = 0) -> list:
+    """L synthetic layers for the verification driver: expert weights, an injected
+    gate matrix [n, E] (the regime's masks, as a router would give them for one
+    draft chunk) and a LayerNorm scale and shift, each layer from its own seed."""
+    layers = []
+    for l in range(L):
+        s = 10_000 * (seed + 1) + l
+        w = make_injected(f"layer{l}", n, n, d_h, E, d_e, dtype, regime, seed=s)
+        ln_gamma = (1.0 + 0.1 * normal(s, 7, (d_h,))).astype(np.float32)
+        ln_beta = (0.1 * normal(s, 8, (d_h,))).astype(np.float32)
+        layers.append({"W_in": w.W_in, "W_out": w.W_out, "gates": w.gates.astype(np.float32),
+                       "ln_gamma": ln_gamma, "ln_beta": ln_beta})
+    return layers
+
+
+def accept_lengths(seed: int, steps: int, n: int, p_accept: float) -> np.ndarray:
+    """Synthetic verification outcomes: each drafted token is accepted with
+    probability p_accept until the first rejection; a step yields the accepted
+    prefix plus the one token the verifier itself produces, so 1 .. n + 1 tokens."""
+    u = _rng(seed, 9).random((steps, n))
+    rejected = u >= p_accept
+    first = np.where(rejected.any(axis=1), rejected.argmax(axis=1), n)
+    return (first + 1).astype(np.int64)
+
+
+def accept_mean(n: int, p_accept: float) -> float:
+    """Closed form of accept_lengths' mean: 1 + sum_{k=1..n} p^k."""
+    p = float(p_accept)
+    return 1.0 + sum(p ** k for k in range(1, n + 1))
