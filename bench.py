@@ -411,6 +411,42 @@ def main():
     torch.cuda.synchronize()
     dense_ms = statistics.median([a.elapsed_time(b) for a, b in dd])
 
+    # the routed decode step, context only: a seeded N(0, 1/d_h) router
+    # (gamma = 1, eps = 2^-23) on the same rotating inputs; the router alone and
+    # router + forward, each as replays of one CUDA graph over the R_COPIES copies
+    W_r = [torch.from_numpy(wl.router_weights(100 + i, E, d_h, "bf16")).to(device=dev, dtype=dt)
+           for i in range(R_COPIES)]
+    gam = torch.ones(E, dtype=torch.float32, device=dev)
+    g_out = torch.empty((T, E), dtype=torch.float32, device=dev)
+    ws_r = bffn.Workspace.for_shapes(T, d_h, E, d_e, n, dt, True, dev)
+
+    def graph_us(fn, reps=8):
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for i in range(R_COPIES):
+                fn(i)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(gr, stream=side):
+                for i in range(R_COPIES):
+                    fn(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            gr.replay()
+            a.record(stream)
+            for _ in range(reps):
+                gr.replay()
+            b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) * 1e3 / (reps * R_COPIES)
+
+    router_us = graph_us(lambda i: bffn.route(bufs[i]["x"], W_r[i], gam, 2.0 ** -23, out=g_out))
+    routed_us = graph_us(lambda i: bffn.forward(bufs[i]["x"], bufs[i]["W_in"], bufs[i]["W_out"], n, W_r=W_r[i],
+                                                gamma=gam, eps=2.0 ** -23, y=bufs[i]["y"], workspace=ws_r))
+
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline()
@@ -449,6 +485,9 @@ def main():
                            "step; a CUDA graph of 8 steps (copies on two side streams, overlapping the "
                            "neighbouring steps' kernels), replayed"},
             "gpu_launches": args.steps,
+            "routed_decode": {"router_us": router_us, "step_us": routed_us,
+                              "what": "router (tensor cores) + single-chunk forward, gates from a seeded "
+                                      "router instead of injected; graph replay"},
             "dense_ffn": {"us": dense_ms * 1e3, "tokens_per_s": T / (dense_ms * 1e-3),
                           "what": "torch bf16: silu(x W_in_cat^T) W_out_cat^T, d_ff = E*d_e"},
             "clocks": clock_info,
