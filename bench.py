@@ -14,12 +14,14 @@ events around each launch give the kernel's own time for the roofline.
 
 The JSON line also carries: the end-to-end number through the public API with
 host buffers (x and gates copied in from pinned memory, y copied out, every
-step), the same-size dense FFN on the GPU (torch bf16 matmuls) for context,
-the HBM roofline fraction on union-expert bytes, the fp64 CPU oracle timed on a
-bounded sample (rank 0, one GPU), and the SM clocks sampled during the run.
+step), the same-size dense FFN on the GPU (torch bf16 matmuls) and the routed
+decode step (router + forward) for context, the HBM roofline fraction on
+union-expert bytes, the fp64 CPU oracle timed on a bounded sample (rank 0, one
+GPU), and the SM clocks sampled during the run.
 
 ``--impl reference`` times the fp64 CPU oracle alone on the same workload and
-metric (there is no runnable upstream implementation).
+metric: the pages ship no runnable implementation of the layer, so the oracle
+(the dense definition in fp64 on the host cores) is the reference arm.
 Multi-GPU (torchrun): independent replicas, one per GPU, no collective on the
 data path (the layer does not shard); weak scaling, max time over ranks.
 """
