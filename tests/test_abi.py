@@ -90,6 +90,20 @@ def test_union_and_route_reject_bad_args(lib):
     assert L.blockffn_route(17, 16, None, 16, 0.0, 32, 64, 16, 1, 16, None) == lib.ERR_INVALID_ARG
 
 
+def test_residual_layernorm_rejects_bad_args(lib):
+    L = lib.lib
+    f = L.blockffn_residual_layernorm
+    assert f(16, 16, 16, 16, 1e-5, 4, 64, 7, 16, None) == lib.ERR_INVALID_ARG          # unknown dtype
+    assert f(16, 16, 16, 16, 1e-5, -1, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG  # T < 0
+    assert f(16, 16, 16, 16, 1e-5, 4, 0, lib.BF16, 16, None) == lib.ERR_INVALID_ARG    # d_h < 1
+    assert f(16, 16, 16, 16, -1.0, 4, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG   # eps < 0
+    assert f(16, 16, 16, 16, float("nan"), 4, 64, lib.F32, 16, None) == lib.ERR_INVALID_ARG
+    assert f(None, 16, 16, 16, 1e-5, 4, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG  # null y
+    assert f(16, 16, 16, None, 1e-5, 4, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG  # null shift
+    # no rows: nothing to do, nothing launched, no pointer needed
+    assert f(None, None, None, None, 1e-5, 0, 64, lib.BF16, None, None) == lib.OK
+
+
 def test_empty_inputs_are_no_ops(lib):
     L = lib.lib
     # T = 0: nothing to do, nothing launched, no pointer needed
