@@ -18,6 +18,19 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(blockffn_[a-z_0-9]+)\s*\(", text)))
 
 
+def test_header_is_plain_c(tmp_path):
+    """The public header compiles on its own as C11 (and C++17), warnings as errors."""
+    import shutil
+    import subprocess
+    for cc, std, ext in (("gcc", "c11", "c"), ("g++", "c++17", "cpp")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not installed")
+        src = tmp_path / f"use.{ext}"
+        src.write_text('#include "blockffn.h"\nint main(void) { return (int)blockffn_version(); }\n')
+        subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-fsyntax-only",
+                        "-I" + os.path.join(ROOT, "include"), str(src)], check=True)
+
+
 @pytest.fixture(scope="module")
 def lib():
     from chunk_sparse_moe_b200 import build
