@@ -82,6 +82,11 @@ int blockffn_version(void);
  * x [T, d_h] and W_r [E, d_h] in dtype dt; b_r [E] fp32 or NULL; gamma [E] fp32;
  * eps >= 0.  gates [T, E] fp32 output.  Requirements: T >= 0, 1 <= E <= 256,
  * d_h >= 1; bf16 additionally d_h % 64 == 0 and E % 16 == 0.
+ * Arithmetic: every sum in a fixed order, so repeated calls give the same bits;
+ * bf16 with d_h % 256 == 0 multiplies on the tensor cores, other shapes on the
+ * CUDA cores (the two orders differ in rounding, not in what they compute).
+ * Stream-ordered; a forward launched right after it may be scheduled early and
+ * waits for it before reading the gates.
  */
 blockffn_status blockffn_route(const void* x, const void* W_r, const float* b_r,
                                const float* gamma, float eps, int T, int d_h, int E,
