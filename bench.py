@@ -49,13 +49,13 @@ UNIT = "tokens/s"
 R_COPIES = 8
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic of the forward kernel from the ncu capture summarised in
-# profiles/union_expert_decode_chunk32.md: (algorithmic bytes, dram__bytes_read.sum
-# + dram__bytes_write.sum) of each captured launch.  The capture covers two of the
-# rotating input copies, so the reported per-launch traffic is their
-# traffic / algorithmic ratio times this run's mean algorithmic bytes.  Empty
-# when the kernel has changed since the capture.
-TRAFFIC_CAPTURE = [(30.679e6, 30.629376e6 + 0), (36.970e6, 36.921600e6 + 6400)]
+# DRAM traffic of the single-chunk forward kernel from an ncu capture of this
+# benchmark's own command (dram__bytes_read.sum + dram__bytes_write.sum of two
+# launches, each on one of the rotating input copies): pairs of (algorithmic
+# bytes, measured bytes) per captured launch.  The reported per-launch traffic is
+# their measured / algorithmic ratio times this run's mean algorithmic bytes.
+# Empty (traffic reported as null) when the kernel has changed since the capture.
+TRAFFIC_CAPTURE = []
 
 
 def peaks():

@@ -369,6 +369,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.skip_unit = g_skip_flag.load();
         da.wait_ns = g_wait_ns.load();
         da.trace = g_trace.load();
+        da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1});
         // A cluster launch cannot also be cooperative; the grid is sized to the
         // pairs that can be resident at once, and every wait is bounded.
         e = launch_forward_decode(da, dmaps, Gd, s);
@@ -414,6 +415,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.wait_ns = g_wait_ns.load();
     a.skip_flag_unit = g_skip_flag.load();
     a.trace = g_trace.load();
+    a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2});
     e = launch_forward_tc(a, maps, G, s);
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "tensor-core forward launch");
 }
@@ -515,6 +517,7 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     da.skip_unit = -1;
     da.wait_ns = g_wait_ns.load();
     da.trace = nullptr;
+    da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)BLOCKFFN_BF16, 0, 3});
     e = launch_forward_decode(da, dmaps, Gd, s);
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "no-allocation forward launch");
 }

@@ -3,6 +3,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <initializer_list>
 #include <cuda_runtime.h>
 
 #include "ptx.cuh"
@@ -30,6 +31,7 @@ enum : int32_t {
     kWaitDrain = 7,      // teardown waiting for its own copies in flight
     kWaitMmaDone = 8,    // teardown waiting for the last MMAs
     kWaitPeers = 9,      // a split unit's block waiting for the other contributors
+    kShapeKey = 10,      // (workspace error) bound to other shapes or another gating mode
 };
 
 // Control block at offset 0 of every forward workspace (256 bytes reserved).
@@ -39,12 +41,37 @@ struct Ctl {
     uint32_t epoch;        // number of completed forward launches (flag stamp)
     uint32_t done;         // thread blocks of the current launch that finished
     uint32_t issued[2];    // by launch parity: blocks that issued their last expert-in load
-    uint32_t pad[58];
+    // The shapes, dtype, gating mode and kernel the workspace's layout was made
+    // for, claimed by the first launch after a reset (0 = not yet bound).  A
+    // launch whose key differs records kErrWorkspace and computes nothing: its
+    // counters and tables would sit at other offsets.
+    unsigned long long shape_key;
+    uint32_t pad[56];
 };
 static_assert(sizeof(Ctl) == 256, "control block is 256 bytes");
 
 __device__ __forceinline__ void record_error(Ctl* ctl, int32_t code, int32_t detail) {
     if (atomicCAS(&ctl->status, 0, code) == 0) atomicExch(&ctl->detail, detail);
+}
+
+// Host-side key of a launch's workspace layout: FNV-1a over the values that
+// decide it.  Never 0 (0 marks an unbound workspace).
+inline unsigned long long shape_key(std::initializer_list<long long> vals) {
+    unsigned long long h = 1469598103934665603ull;
+    for (long long v : vals) {
+        for (int b = 0; b < 8; ++b) {
+            h ^= (unsigned long long)((v >> (8 * b)) & 0xff);
+            h *= 1099511628211ull;
+        }
+    }
+    return h | 1ull;
+}
+
+// Claim the workspace for this launch's key, or find it bound to the same key.
+// Returns the previous key; the caller compares (one atomic, issued beside the
+// prologue's other control-block accesses so its latency overlaps theirs).
+__device__ __forceinline__ unsigned long long claim_shape_key(Ctl* ctl, unsigned long long key) {
+    return atomicCAS(&ctl->shape_key, 0ull, key);
 }
 
 // Spin on an mbarrier phase for at most limit_ns.  Gives up early when another

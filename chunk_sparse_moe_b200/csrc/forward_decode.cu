@@ -273,16 +273,20 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // acquire: the read is done before this block's count below is seen
         const uint32_t ep0 = ld_acquire_gpu(&a.ctl->epoch);
         if (blockIdx.x == 0) a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;   // the next launch's counter
-        sh.abort = st0 != 0;
         sh.epoch = ep0;
         // The last block to read the launch counter advances it for the next
         // launch (every block of this one has read it by then; the next launch
         // sees the new value because it reads it only after this one has
         // completed: stream order, or its griddep_wait).
-        if (atomicAdd(&a.ctl->done, 1u) == (uint32_t)(gridDim.x - 1)) {
+        const uint32_t done0 = atomicAdd(&a.ctl->done, 1u);
+        const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
+        if (done0 == (uint32_t)(gridDim.x - 1)) {
             a.ctl->done = 0u;
             a.ctl->epoch = ep0 + 1u;
         }
+        const bool key_ok = key0 == 0ull || key0 == a.shape_key;
+        if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
+        sh.abort = st0 != 0 || !key_ok;
     }
     if (warp >= 3) {
         // the chunk's union, ascending (warps 3-6 take 32-expert groups; all of a
@@ -320,8 +324,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     const int nBt = wk.bHi - wk.bLo;                 // expert-out tiles per owned row tile
     const int totB = P > 0 ? wk.nRT * nBt : 0;        // this block's expert-out tiles
     const bool doB = P > 0 && wk.nRT > 0;             // this cluster sums expert-out row tiles
-    if (threadIdx.x == 0 && doB) {
+    if (threadIdx.x == 0 && doB && !sh.abort) {
         // the first expert-out reduction: 3 quadrant partials of 32 rows x N tokens
+        // (not armed by a launch that computes nothing, whose teardown would
+        // otherwise wait for bytes nobody sends)
         mbar_arrive_expect_tx(&sh.recvB, 3u * 32u * N * 4u);
         sh.pendB = 0;
     }

@@ -6,13 +6,18 @@
 // (non-gated Swish experts).
 //
 // The fp32 workload needs a relative L2 error of 1e-5, which TF32 tensor cores
-// cannot give, so this path stays on FFMA.  Two kernels:
-//   A: one block per (chunk, union expert) pair: h'[p, j, :] =
-//      bit_j ? g[t,e] * Swish(W_in_e x_t) : 0 for the chunk's tokens.  A masked
-//      token's activation is exactly zero whether or not it is computed, so the
-//      block skips the dot products of masked tokens.
-//   B: y[t, i] = sum over the chunk's union experts, ascending, of
-//      W_out_e[i, :] . h'[p, j, :], one thread per output element, a fixed order.
+// cannot give, so this path stays on FFMA.  Two kernels, both staging coalesced
+// 64 x 64 tiles of the weights and of the chunk's activations in shared memory;
+// a lane owns one token of the chunk and a warp eight output rows:
+//   A: one block per (chunk, union expert) pair at a time:
+//        h[j, r]  = sum_k W_in_e[r, k] x[t_j, k]        for every token j of the chunk
+//        h'[j, r] = bit_j ? g[t_j, e] * Swish(h[j, r]) : 0
+//      Every token of the chunk is computed and the mask applied afterwards (a
+//      select, so a masked token gives exactly 0), as the method states.
+//   B: one block per (64 rows of y, chunk):
+//        y[t_j, i] = sum over the chunk's union experts, ascending, of
+//                    sum_q W_out_e[i, q] h'[p, j, q]
+//      each output's sum running sequentially over (expert, q): a fixed order.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -20,51 +25,106 @@
 
 namespace bffn {
 
-__global__ void __launch_bounds__(256) expert_in_f32_kernel(
+constexpr int kF32Tile = 64;       // rows and k per staged tile
+constexpr int kF32Threads = 256;   // 8 warps x 8 rows
+
+__global__ void __launch_bounds__(kF32Threads) expert_in_f32_kernel(
     const float* __restrict__ x, const float* __restrict__ gates, const float* __restrict__ W_in,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ pair_ce,
     const uint32_t* __restrict__ tmask, int T, int d_h, int E, int d_e, int n, int C,
     float* __restrict__ hbuf) {
+    __shared__ float sw[kF32Tile][kF32Tile + 1];   // [row][k]
+    __shared__ float sx[32][kF32Tile + 1];         // [token][k]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = offsets[C];
     for (int p = blockIdx.x; p < P; p += gridDim.x) {
         const int ce = pair_ce[p];
         const int c = ce >> 8, e = ce & 255;
         const uint32_t bits = tmask[(size_t)c * E + e];
-        for (int o = threadIdx.x; o < n * d_e; o += blockDim.x) {
-            const int j = o / d_e, row = o % d_e;
-            const int t = c * n + j;
-            float out = 0.f;
-            if (t < T && ((bits >> j) & 1u)) {
-                const float* w = W_in + ((size_t)e * d_e + row) * d_h;
-                const float* xt = x + (size_t)t * d_h;
-                float z = 0.f;
-                for (int k = 0; k < d_h; ++k) z = fmaf(__ldg(w + k), __ldg(xt + k), z);
-                const float sw = z / (1.0f + expf(-z));
-                out = gates[(size_t)t * E + e] * sw;
+        const int t = c * n + lane;                       // this lane's token
+        const bool live = lane < n && t < T;              // a token of the chunk
+        const float g = live ? gates[(size_t)t * E + e] : 0.f;
+        for (int r0 = 0; r0 < d_e; r0 += kF32Tile) {
+            float acc[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+            for (int k0 = 0; k0 < d_h; k0 += kF32Tile) {
+                __syncthreads();
+                for (int i = threadIdx.x; i < kF32Tile * kF32Tile; i += kF32Threads) {
+                    const int r = i / kF32Tile, k = i % kF32Tile;
+                    sw[r][k] = (r0 + r < d_e && k0 + k < d_h)
+                                   ? __ldg(W_in + ((size_t)e * d_e + r0 + r) * d_h + k0 + k) : 0.f;
+                }
+                for (int i = threadIdx.x; i < 32 * kF32Tile; i += kF32Threads) {
+                    const int j = i / kF32Tile, k = i % kF32Tile;
+                    const int tj = c * n + j;
+                    sx[j][k] = (j < n && tj < T && k0 + k < d_h) ? __ldg(x + (size_t)tj * d_h + k0 + k) : 0.f;
+                }
+                __syncthreads();
+#pragma unroll 4
+                for (int k = 0; k < kF32Tile; ++k) {
+                    const float xv = sx[lane][k];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) acc[u] = fmaf(sw[warp * 8 + u][k], xv, acc[u]);
+                }
             }
-            hbuf[((size_t)p * n + j) * d_e + row] = out;
+            if (lane < n) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = r0 + warp * 8 + u;
+                    if (r >= d_e) break;
+                    const float z = acc[u];
+                    const float act = g * (z / (1.0f + expf(-z)));
+                    hbuf[((size_t)p * n + lane) * d_e + r] = (live && ((bits >> lane) & 1u)) ? act : 0.f;
+                }
+            }
         }
     }
 }
 
-__global__ void __launch_bounds__(128) expert_out_f32_kernel(
+__global__ void __launch_bounds__(kF32Threads) expert_out_f32_kernel(
     const float* __restrict__ W_out, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ pair_ce,
     const float* __restrict__ hbuf, int T, int d_h, int d_e, int n, float* __restrict__ y) {
+    __shared__ float sw[kF32Tile][kF32Tile + 1];   // [row i][q]
+    __shared__ float sh[32][kF32Tile + 1];         // [token][q]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.y;
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= d_h) return;
+    const int i0 = blockIdx.x * kF32Tile;
     const int cnt = counts[c], off = offsets[c];
     const int t0 = c * n, nt = min(n, T - t0);
-    for (int j = 0; j < nt; ++j) {
-        float acc = 0.f;
-        for (int s = 0; s < cnt; ++s) {
-            const int e = pair_ce[off + s] & 255;
-            const float* w = W_out + ((size_t)e * d_h + i) * d_e;
-            const float* h = hbuf + ((size_t)(off + s) * n + j) * d_e;
-            for (int q = 0; q < d_e; ++q) acc = fmaf(__ldg(w + q), h[q], acc);
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+    for (int s = 0; s < cnt; ++s) {
+        const int e = pair_ce[off + s] & 255;
+        const float* hp = hbuf + (size_t)(off + s) * n * d_e;
+        for (int q0 = 0; q0 < d_e; q0 += kF32Tile) {
+            __syncthreads();
+            for (int i = threadIdx.x; i < kF32Tile * kF32Tile; i += kF32Threads) {
+                const int r = i / kF32Tile, q = i % kF32Tile;
+                sw[r][q] = (i0 + r < d_h && q0 + q < d_e)
+                               ? __ldg(W_out + ((size_t)e * d_h + i0 + r) * d_e + q0 + q) : 0.f;
+            }
+            for (int i = threadIdx.x; i < 32 * kF32Tile; i += kF32Threads) {
+                const int j = i / kF32Tile, q = i % kF32Tile;
+                sh[j][q] = (j < nt && q0 + q < d_e) ? hp[(size_t)j * d_e + q0 + q] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int q = 0; q < kF32Tile; ++q) {
+                const float hv = sh[lane][q];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] = fmaf(sw[warp * 8 + u][q], hv, acc[u]);
+            }
         }
-        y[(size_t)(t0 + j) * d_h + i] = acc;
+    }
+    if (lane < nt) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + warp * 8 + u;
+            if (i < d_h) y[(size_t)(t0 + lane) * d_h + i] = acc[u];
+        }
     }
 }
 
@@ -75,15 +135,16 @@ cudaError_t launch_forward_f32(const float* x, const float* gates, const float* 
                                cudaStream_t s) {
     const int C = (T + n - 1) / n;
     if (C == 0) return cudaSuccess;
+    if (C > 65535) return cudaErrorInvalidValue;
     const long long pmax = (long long)C * E;
     const int gridA = (int)(pmax < 8LL * num_sms ? pmax : 8LL * num_sms);
-    expert_in_f32_kernel<<<gridA, 256, 0, s>>>(x, gates, W_in, offsets, pair_ce, tmask, T, d_h,
-                                               E, d_e, n, C, hbuf);
+    expert_in_f32_kernel<<<gridA, kF32Threads, 0, s>>>(x, gates, W_in, offsets, pair_ce, tmask, T, d_h,
+                                                       E, d_e, n, C, hbuf);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    dim3 gridB((d_h + 127) / 128, C);
-    expert_out_f32_kernel<<<gridB, 128, 0, s>>>(W_out, counts, offsets, pair_ce, hbuf, T, d_h,
-                                                d_e, n, y);
+    dim3 gridB((d_h + kF32Tile - 1) / kF32Tile, C);
+    expert_out_f32_kernel<<<gridB, kF32Threads, 0, s>>>(W_out, counts, offsets, pair_ce, hbuf, T, d_h,
+                                                        d_e, n, y);
     return cudaGetLastError();
 }
 

@@ -242,7 +242,10 @@ union_expert_forward_tc(const __grid_constant__ CUtensorMap tm_x,
         // written by earlier launches only: plain L2 loads, issued together
         const int32_t st0 = __ldcg(&a.ctl->status);
         const uint32_t ep0 = __ldcg(&a.ctl->epoch);
-        sh.abort = st0 != 0;
+        const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
+        const bool key_ok = key0 == 0ull || key0 == a.shape_key;
+        if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
+        sh.abort = st0 != 0 || !key_ok;
         sh.epoch = ep0;
         BFFN_TRACE(kTrCtlLoaded);
         prefetch_tmap(&tm_x);

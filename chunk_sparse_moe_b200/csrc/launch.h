@@ -64,6 +64,7 @@ struct TcArgs {
     int skip_flag_unit;   // test support: unit whose h' is never announced ready (-1: off)
     unsigned long long* trace;   // optional [grid][16] globaltimer stamps (nullptr: off)
     unsigned long long wait_ns;
+    unsigned long long shape_key;   // the workspace layout this launch expects (Ctl::shape_key)
 };
 
 // maps: x, W_in, W_out (2-D, bf16, 128-byte swizzle, boxes {64,N}, {64,128}, {64,128})
@@ -86,6 +87,7 @@ struct DcArgs {
     int skip_unit;            // test support: expert-in half never counted in (-1: off)
     unsigned long long wait_ns;
     unsigned long long* trace;   // optional [grid][64] globaltimer stamps
+    unsigned long long shape_key;   // the workspace layout this launch expects (Ctl::shape_key)
 };
 // maps: x [T, d_h] (box N rows), W_in [E*d_e, d_h] and W_out [E*d_h, d_e] (box 128
 // rows), h' [E*N, d_e] (box N rows): 3-D {64, rows, column block} boxes of two

@@ -157,7 +157,11 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  * fully overwritten (rows of tokens with no active expert are exact zeros).
  * workspace: ws_bytes >= blockffn_forward_workspace_bytes(...), reset once with
  * blockffn_workspace_reset; it carries state between calls (never share one
- * workspace between calls that may overlap on the GPU).
+ * workspace between calls that may overlap on the GPU).  The first call after a
+ * reset binds the workspace to its (T, d_h, E, d_e, n, dt, gating mode); a later
+ * call with any of these different records BLOCKFFN_ERR_WORKSPACE in the status
+ * word (blockffn_get_device_status, detail 10) and computes nothing.  Reset the
+ * workspace, or use another one, to change them.
  * Requirements: T >= 0, 1 <= n <= 32, 1 <= E <= 256;
  *   bf16: d_h % 128 == 0, d_e % 128 == 0, d_e <= 512, E % 16 == 0 when routed;
  *   fp32: any d_h, d_e >= 1.
@@ -207,7 +211,8 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
  * blockffn_get_device_status -- synchronize stream, then read the device status
  * word of a workspace: BLOCKFFN_OK, or the first device-side error recorded
  * (BLOCKFFN_ERR_TIMEOUT, BLOCKFFN_ERR_WORKSPACE).  detail (may be NULL) receives
- * a code naming the wait that ran out.  Returns BLOCKFFN_ERR_CUDA if the
+ * a code naming the wait that ran out (1-9), or 10 for a workspace bound to
+ * other shapes or another gating mode.  Returns BLOCKFFN_ERR_CUDA if the
  * synchronization itself failed.
  */
 blockffn_status blockffn_get_device_status(const void* workspace, void* stream,

@@ -157,6 +157,59 @@ def test_forward_partly_empty_chunks(bffn):
     assert_close(y, oracle_y(w, g), "bf16", "mixed")
 
 
+@pytest.mark.parametrize("bias", [-0.8, None])
+def test_forward_routed_single_chunk_bf16(bffn, bias):
+    """The routed decode step: tensor-core router, then the single-chunk kernel
+    launched as its programmatic dependent reading the gates from the workspace
+    (T = n = 32, d_h 2048, E 64).  Masks as in the router tests; y against the
+    oracle given the GPU's gates."""
+    w = wl.make_routed("routed32", 32, 32, 2048, 64, 128, "bf16", seed=31, bias_shift=bias)
+    g_chk = _check_route(bffn, w)
+    y, g = run_gpu(w)
+    assert np.array_equal(g, g_chk), "the forward's router and blockffn_route disagree"
+    assert_close(y, oracle_y(w, g), "bf16", f"routed single chunk bias {bias}")
+
+
+@pytest.mark.parametrize("T,n,d_h,E,d_e", [
+    (32, 32, 256, 16, 256),     # two 128-row tiles per expert (MT = 2)
+    (20, 32, 512, 16, 512),     # MT = 4, short chunk
+    (32, 32, 2048, 16, 384),    # MT = 3 at the benchmark's d_h
+    (8, 8, 1024, 32, 256),      # N = 16 tokens per MMA, MT = 2
+])
+def test_forward_single_chunk_wide_experts(bffn, T, n, d_h, E, d_e):
+    """The single-chunk kernel (T <= n, d_h % 256 == 0) with d_e > 128: several
+    expert-in row tiles per expert and several k-block pairs per expert-out tile."""
+    w = wl.make_injected("wide", T, n, d_h, E, d_e, "bf16", "markov80", seed=T + d_e)
+    y, g = run_gpu(w)
+    assert_close(y, oracle_y(w, g), "bf16", f"single chunk T{T} n{n} d_h{d_h} E{E} d_e{d_e}")
+
+
+def test_workspace_bound_to_its_shapes(bffn):
+    """A workspace is bound to the shapes and gating mode of its first call after a
+    reset: a call with other shapes is refused on the device (status
+    BLOCKFFN_ERR_WORKSPACE, detail 10) and writes nothing; after a reset the new
+    shapes compute correctly."""
+    ERR_WORKSPACE, SHAPE_KEY = 5, 10
+    big = wl.make_routed("bind", 96, 32, 2048, 64, 128, "bf16", seed=7, bias_shift=-0.8)
+    small = wl.chunk32()
+    nb = max(bffn.workspace_bytes(96, 2048, 64, 128, 32, torch.bfloat16, True),
+             bffn.workspace_bytes(32, 2048, 64, 128, 32, torch.bfloat16, False))
+    ws = bffn.Workspace(nb)
+    y, g = run_gpu(big, ws)
+    assert_close(y, oracle_y(big, g), "bf16", "first binding")
+    assert bffn.device_status(ws) == (0, 0)
+    x = dev(small.x, torch.bfloat16)
+    W_in, W_out = dev(small.W_in, torch.bfloat16), dev(small.W_out, torch.bfloat16)
+    yy = torch.full((32, 2048), 3.0, dtype=torch.bfloat16, device="cuda")
+    bffn.forward(x, W_in, W_out, 32, gates=dev(small.gates, torch.float32), y=yy, workspace=ws)
+    assert bffn.device_status(ws) == (ERR_WORKSPACE, SHAPE_KEY)
+    assert torch.all(yy == 3.0)
+    ws.reset()
+    y2, g2 = run_gpu(small, ws)
+    assert_close(y2, oracle_y(small, g2), "bf16", "after reset")
+    assert bffn.device_status(ws) == (0, 0)
+
+
 def test_forward_router_bf16_small(bffn):
     w = wl.make_routed("r", 100, 32, 256, 16, 128, "bf16", seed=5, bias_shift=-0.8, ar_rho=0.95)
     y, g = run_gpu(w)
@@ -284,26 +337,44 @@ def test_workload_chunk32_full(bffn):
     assert_close(y, oracle.forward_dense(w.x, g, w.W_in, w.W_out), "bf16", "chunk32")
 
 
-def test_workload_batch16_sampled_chunks(bffn):
+def test_workload_batch16_all_chunks(bffn):
     w = wl.batch16()
     y, g = run_gpu(w)
-    tok = chunk_tokens(w, [0, 7, 15])
-    assert_close(y[tok], oracle_y(w, g, tok), "bf16", "batch16")
+    assert_close(y, oracle_y(w, g), "bf16", "batch16")
+    for c in range(w.C):   # and chunk by chunk, so one bad chunk cannot hide in the norm
+        tok = chunk_tokens(w, [c])
+        assert_close(y[tok], oracle_y(w, g, tok), "bf16", f"batch16 chunk {c}")
 
 
-def test_workload_seq4096_sampled_chunks(bffn):
+def test_workload_seq4096_all_chunks(bffn):
+    """Router + union + forward over 4096 tokens; every chunk against the oracle
+    (which visits only each chunk's union experts), given the GPU's gates."""
     w = wl.seq4096()
     y, g = run_gpu(w)
-    tok = chunk_tokens(w, [0, 64, 127])
-    assert_close(y[tok], oracle_y(w, g, tok), "bf16", "seq4096")
+    ref = oracle_y(w, g)
+    assert_close(y, ref, "bf16", "seq4096")
+    for c in range(w.C):
+        tok = chunk_tokens(w, [c])
+        assert_close(y[tok], ref[tok], "bf16", f"seq4096 chunk {c}")
     # every row: zero exactly where no expert is active
     assert np.array_equal(np.any(y != 0, axis=1), np.any(g != 0, axis=1))
 
 
 @pytest.mark.parametrize("n", wl.SWEEP_CHUNKS)
 @pytest.mark.parametrize("regime", wl.SWEEP_REGIMES)
-def test_workload_sweep_first_chunk(bffn, n, regime):
-    """d_h=4096, E=128: one decode-step call on the sequence's first chunk."""
-    w = wl.sweep(n, regime, T=n)
-    y, g = run_gpu(w)
-    assert_close(y, oracle_y(w, g), "bf16", f"sweep n{n} {regime}")
+def test_workload_sweep_chunks(bffn, n, regime):
+    """d_h=4096, E=128: decode-step calls (one chunk each, as the sweep runs them)
+    on chunks spread over the first 1024 tokens of the sequence."""
+    T = 1024
+    w = wl.sweep(n, regime, T=T)
+    C = (T + n - 1) // n
+    W_in, W_out = dev(w.W_in, torch.bfloat16), dev(w.W_out, torch.bfloat16)
+    ws = bffn.Workspace.for_shapes(n, w.d_h, w.E, w.d_e, n, torch.bfloat16, False)
+    for c in sorted({0, C // 3, (2 * C) // 3, C - 1}):
+        sl = slice(c * n, (c + 1) * n)
+        y = bffn.forward(dev(w.x[sl], torch.bfloat16), W_in, W_out, n,
+                         gates=dev(w.gates[sl], torch.float32), workspace=ws)
+        torch.cuda.synchronize()
+        ref = oracle.forward_chunk_union(w.x[sl], w.gates[sl].astype(np.float64), w.W_in, w.W_out, n)
+        assert_close(to_np64(y), ref, "bf16", f"sweep n{n} {regime} chunk {c}")
+    assert bffn.device_status(ws) == (0, 0)

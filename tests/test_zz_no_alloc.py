@@ -33,14 +33,19 @@ def _noalloc(lib, x, g, W_in, W_out, n, y):
                                         torch.cuda.current_stream().cuda_stream)
 
 
-def test_noalloc_matches_forward_on_two_calls():
+@pytest.mark.parametrize("T,n,d_e", [(32, 32, 128), (8, 8, 128), (5, 32, 128), (32, 32, 256)])
+def test_noalloc_matches_forward_on_two_calls(T, n, d_e):
+    """Full chunks, the 16-token variant (n <= 16), a short chunk and wider
+    experts, each on two calls in a row with different inputs."""
     bffn = require_cuda()
     from chunk_sparse_moe_b200 import _lib
-    base = wl.chunk32()
+    d_h, E = 2048, 64
+    base = wl.make_injected("noalloc", T, n, d_h, E, d_e, "bf16", "markov80", seed=T + n + d_e)
     weights = (base.W_in, base.W_out)
     W_in, W_out = dev(base.W_in, torch.bfloat16), dev(base.W_out, torch.bfloat16)
-    for call, x_seed in enumerate((0, 5)):
-        w = wl.chunk32(weights=weights, x_seed=x_seed)
+    for call, x_seed in enumerate((3, 5)):
+        w = wl.make_injected("noalloc", T, n, d_h, E, d_e, "bf16", "markov80", seed=T + n + d_e,
+                             weights=weights, x_seed=x_seed)
         x, g = dev(w.x, torch.bfloat16), dev(w.gates, torch.float32)
         y_ref = bffn.forward(x, W_in, W_out, w.n, gates=g)          # caller workspace
         y = torch.full_like(y_ref, float("nan"))
@@ -55,6 +60,26 @@ def test_noalloc_matches_forward_on_two_calls():
         # and against the oracle directly
         ref = oracle_y(w, w.gates.astype(np.float64))
         assert rel_l2(a, ref) <= BF16_REL_L2
+
+
+def test_noalloc_empty_union_writes_zeros():
+    """All gates zero after a call that left h' and counters in the shared
+    scratch: y is written as exact zeros, then a normal call is correct again."""
+    require_cuda()
+    from chunk_sparse_moe_b200 import _lib
+    w = wl.chunk32()
+    x, W_in, W_out = (dev(a, torch.bfloat16) for a in (w.x, w.W_in, w.W_out))
+    g = dev(w.gates, torch.float32)
+    y = torch.empty((w.T, w.d_h), dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(_lib.lib, x, g, W_in, W_out, w.n, y) == OK
+    y0 = torch.full_like(y, float("nan"))
+    assert _noalloc(_lib.lib, x, torch.zeros_like(g), W_in, W_out, w.n, y0) == OK
+    torch.cuda.synchronize()
+    assert not torch.any(y0 != 0) and not torch.any(torch.isnan(y0))
+    y1 = torch.full_like(y, float("nan"))
+    assert _noalloc(_lib.lib, x, g, W_in, W_out, w.n, y1) == OK
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y)
 
 
 def test_noalloc_refuses_what_does_not_fit():
