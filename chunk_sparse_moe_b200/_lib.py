@@ -38,6 +38,7 @@ SIGNATURES = {
                                                     c_int]),
     "blockffn_workspace_reset": (c_int, [c_void_p, c_size_t, c_void_p]),
     "blockffn_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float,
+                                 c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                  c_void_p, c_void_p, c_size_t, c_void_p]),
     "blockffn_get_device_status": (c_int, [c_void_p, c_void_p, c_int32_p]),

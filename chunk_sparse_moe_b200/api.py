@@ -147,15 +147,20 @@ def forward(x: torch.Tensor, W_in: torch.Tensor, W_out: torch.Tensor, n: int,
             gates: Optional[torch.Tensor] = None, W_r: Optional[torch.Tensor] = None,
             b_r: Optional[torch.Tensor] = None, gamma: Optional[torch.Tensor] = None,
             eps: float = 2.0 ** -23, y: Optional[torch.Tensor] = None,
-            workspace: Optional[Workspace] = None) -> torch.Tensor:
-    """y [T, d_h] = sum over each chunk's union experts of gate * W_out_e Swish(W_in_e x)."""
+            workspace: Optional[Workspace] = None, union=None) -> torch.Tensor:
+    """y [T, d_h] = sum over each chunk's union experts of gate * W_out_e Swish(W_in_e x).
+
+    ``union``: optional (counts, idx, tmask) as ``chunk_union`` returns them for
+    these gates and n; the forward then uses them instead of forming the union."""
     T, d_h = x.shape
     E, d_e, _ = W_in.shape
     if y is None:
         y = torch.empty((T, d_h), dtype=x.dtype, device=x.device)
     if workspace is None:
         workspace = Workspace.for_shapes(T, d_h, E, d_e, n, x.dtype, gates is None, x.device)
+    counts, idx, tmask = union if union is not None else (None, None, None)
     st = lib.blockffn_forward(_ptr(x), _ptr(gates), _ptr(W_r), _ptr(b_r), _ptr(gamma), float(eps),
+                              _ptr(counts), _ptr(idx), _ptr(tmask),
                               _ptr(W_in), _ptr(W_out), T, d_h, E, d_e, n, _dtype_code(x),
                               _ptr(y), workspace.buf.data_ptr(), workspace.nbytes, _stream())
     _check(st, "blockffn_forward")

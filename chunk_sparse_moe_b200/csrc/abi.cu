@@ -118,51 +118,99 @@ bool make_map_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Which kernel computes a forward call.
+enum class Path { F32, Decode, Group };
+
+// Workspace layout of one forward call (byte offsets; 0 = not used by the path).
 struct Layout {
-    size_t ctl, counts, offsets, idx, tmask, pair_ce, gates, cntA, readyA, cntB, partA, partB, hbuf;
+    Path path;
+    size_t ctl, counts, offsets, idx, tmask, pair_ce, gcounts, goffsets, gpair, gates;
+    size_t cntA, readyA, cntB, partA, partB, hbuf;
     size_t total;
-    int C, N, MT, RT, KB, KBe;
-    long long Pmax;
+    int C;               // chunks
+    int N;               // tokens per MMA
+    int NG, NT, NGr;     // group kernel: chunks and tokens per group, groups
+    int MT, RT, KB, KBe;
+    long long Pmax;      // pairs the tables can hold
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-bool make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_router, int G,
-                 Layout& L) {
+int decode_clusters_current() {
+    static int cache[64];
+    static std::once_flag once[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    std::call_once(once[dev], [dev]() { cache[dev] = decode_max_clusters(); });
+    return cache[dev];
+}
+
+// The single-chunk kernel's grid (4 blocks per cluster), or 0 when it cannot run
+// these shapes here.
+int decode_grid(int C, int d_h, int E, int G) {
+    if (C != 1 || (d_h / 64) % 4 != 0 || E > 256) return 0;
+    int ncl = decode_clusters_current();
+    if (ncl > G / 4) ncl = G / 4;
+    if (ncl <= 0 || 4 * ncl > 160) return 0;
+    return 4 * ncl;
+}
+
+void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_router, int G, Layout& L) {
     L.C = (T + n - 1) / n;
-    L.N = bf16 ? (n <= 16 ? 16 : 32) : n;
     L.MT = bf16 ? d_e / 128 : 1;
     L.RT = bf16 ? d_h / 128 : 1;
     L.KB = bf16 ? d_h / 64 : 1;
     L.KBe = bf16 ? d_e / 64 : 1;
-    L.Pmax = (long long)L.C * E;
+    L.path = !bf16 ? Path::F32 : (decode_grid(L.C, d_h, E, G) > 0 ? Path::Decode : Path::Group);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off = align_up(off + (bytes > 0 ? bytes : 1), 256);
         return o;
     };
-    const size_t C = (size_t)L.C, Pm = (size_t)L.Pmax;
+    L.ctl = L.counts = L.offsets = L.idx = L.tmask = L.pair_ce = L.gcounts = L.goffsets = L.gpair = 0;
+    L.gates = L.cntA = L.readyA = L.cntB = L.partA = L.partB = L.hbuf = 0;
+    L.NG = L.NT = L.NGr = 0;
+    const size_t C = (size_t)L.C;
     L.ctl = take(sizeof(Ctl));
-    L.counts = take(C * 4);
-    L.offsets = take((C + 1) * 4);
-    L.idx = take(C * E * 4);
-    L.tmask = take(C * E * 4);
-    L.pair_ce = take(Pm * 4);
-    L.gates = with_router ? take((size_t)T * E * 4) : 0;
-    if (bf16) {
+    if (with_router) L.gates = take((size_t)T * E * 4);
+    if (L.path == Path::F32) {
+        L.N = n;
+        L.Pmax = (long long)L.C * E;
+        L.counts = take(C * 4);
+        L.offsets = take((C + 1) * 4);
+        L.idx = take(C * E * 4);
+        L.tmask = take(C * E * 4);
+        L.pair_ce = take((size_t)L.Pmax * 4);
+        L.hbuf = take((size_t)L.Pmax * n * d_e * 4);
+    } else if (L.path == Path::Decode) {
+        // the single-chunk kernel forms the union itself: counters and h' only
+        L.N = n <= 16 ? 16 : 32;
+        L.Pmax = E;
+        L.readyA = take(2 * (size_t)E * 4);
+        L.hbuf = take((size_t)E * L.N * d_e * 2);
+    } else {
+        // groups of whole chunks, N = 128 tokens per MMA for short inputs, else 256
+        L.N = T <= 128 ? 128 : 256;
+        L.NG = L.N / n;
+        L.NT = L.NG * n;
+        L.NGr = (L.C + L.NG - 1) / L.NG;
+        L.Pmax = (long long)L.NGr * E;
+        const size_t NGr = (size_t)L.NGr, Pm = (size_t)L.Pmax;
+        L.counts = take(C * 4);
+        L.idx = take(C * E * 4);
+        L.tmask = take(C * E * 4);
+        L.gcounts = take(NGr * 4);
+        L.goffsets = take((NGr + 1) * 4);
+        L.gpair = take(Pm * 4);
         L.cntA = take(2 * Pm * L.MT * 4);
         L.readyA = take(2 * Pm * L.MT * 4);
-        L.cntB = take(2 * C * L.RT * 4);
+        L.cntB = take(2 * NGr * L.RT * 4);
         L.partA = take((size_t)G * 2 * L.N * 128 * 4);
         L.partB = take((size_t)G * 2 * L.N * 128 * 4);
         L.hbuf = take(Pm * L.N * d_e * 2);
-    } else {
-        L.cntA = L.readyA = L.cntB = L.partA = L.partB = 0;
-        L.hbuf = take(Pm * n * d_e * 4);
     }
     L.total = off;
-    return true;
 }
 
 blockffn_status check_shapes(int T, int d_h, int E, int d_e, int n, blockffn_dtype dt) {
@@ -207,7 +255,7 @@ const char* blockffn_status_string(blockffn_status s) {
 
 const char* blockffn_last_error_message(void) { return g_msg; }
 
-int blockffn_version(void) { return 100; }
+int blockffn_version(void) { return 20000; }
 
 void blockffn_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns > 0 ? ns : 1); }
 
@@ -276,6 +324,7 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
 
 blockffn_status blockffn_forward(const void* x, const float* gates, const void* W_r,
                                  const float* b_r, const float* gamma, float eps,
+                                 const int32_t* counts, const int32_t* idx, const uint32_t* tmask,
                                  const void* W_in, const void* W_out, int T, int d_h, int E,
                                  int d_e, int n, blockffn_dtype dt, void* y, void* workspace,
                                  size_t ws_bytes, void* stream) {
@@ -283,18 +332,25 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     if (st != BLOCKFFN_OK) return st;
     if (T == 0) return BLOCKFFN_OK;   // nothing to compute (empty tensors may be NULL)
     const bool routed = gates == nullptr;
+    const int ntab = (counts != nullptr) + (idx != nullptr) + (tmask != nullptr);
+    if (ntab != 0 && ntab != 3)
+        return fail(BLOCKFFN_ERR_INVALID_ARG, "pass all of counts, idx and tmask, or none of them");
+    const bool tables = ntab == 3;
     if (routed) {
         if (!W_r || !gamma) return fail(BLOCKFFN_ERR_INVALID_ARG, "no gates: W_r and gamma are required");
         if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(BLOCKFFN_ERR_INVALID_ARG, "eps must be finite and >= 0");
         if (dt == BLOCKFFN_BF16 && E % 16 != 0)
             return fail(BLOCKFFN_ERR_UNSUPPORTED, "bf16 router needs E %% 16 == 0");
+        if (tables)
+            return fail(BLOCKFFN_ERR_INVALID_ARG, "union tables can only come with injected gates");
     } else if (W_r || b_r || gamma) {
         return fail(BLOCKFFN_ERR_INVALID_ARG, "pass either gates or router weights, not both");
     }
     if (!x || !W_in || !W_out || !y || !workspace) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(x) || !aligned16(W_in) || !aligned16(W_out) || !aligned16(y) ||
         !aligned16(workspace) || (gates && !aligned16(gates)) || (W_r && !aligned16(W_r)) ||
-        (gamma && !aligned16(gamma)) || (b_r && !aligned16(b_r)))
+        (gamma && !aligned16(gamma)) || (b_r && !aligned16(b_r)) || (counts && !aligned16(counts)) ||
+        (idx && !aligned16(idx)) || (tmask && !aligned16(tmask)))
         return fail(BLOCKFFN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
     const int G = num_sms_current();
     if (G <= 0) return fail(BLOCKFFN_ERR_CUDA, "no current CUDA device");
@@ -305,6 +361,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         return fail(BLOCKFFN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, L.total);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
+    Ctl* ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
     cudaError_t e;
 
     const float* g = gates;
@@ -314,37 +371,29 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         if (e != cudaSuccess) return cuda_fail(e, "route launch");
         g = gw;
     }
-    int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
-    int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
-    int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
-    uint32_t* tmask = reinterpret_cast<uint32_t*>(ws + L.tmask);
-    int32_t* pair_ce = reinterpret_cast<int32_t*>(ws + L.pair_ce);
+    // the union tables: the caller's (checked on the device against its token
+    // masks), or the workspace's, computed from the gates
+    int32_t* t_counts = tables ? const_cast<int32_t*>(counts) : reinterpret_cast<int32_t*>(ws + L.counts);
+    int32_t* t_idx = tables ? const_cast<int32_t*>(idx) : reinterpret_cast<int32_t*>(ws + L.idx);
+    uint32_t* t_tmask = tables ? const_cast<uint32_t*>(tmask) : reinterpret_cast<uint32_t*>(ws + L.tmask);
 
-    if (!bf16) {
-        e = launch_chunk_union_plan(g, T, E, n, counts, idx, tmask, offsets, pair_ce, y, d_h, 4, s);
+    if (L.path == Path::F32) {
+        int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+        int32_t* pair_ce = reinterpret_cast<int32_t*>(ws + L.pair_ce);
+        e = launch_chunk_union_plan(g, T, E, n, t_counts, t_idx, t_tmask, !tables, ctl, offsets, pair_ce, y,
+                                    d_h, 4, s);
         if (e != cudaSuccess) return cuda_fail(e, "union launch");
         e = launch_forward_f32(static_cast<const float*>(x), g, static_cast<const float*>(W_in),
-                               static_cast<const float*>(W_out), counts, offsets, pair_ce, tmask,
+                               static_cast<const float*>(W_out), t_counts, offsets, pair_ce, t_tmask, ctl,
                                reinterpret_cast<float*>(ws + L.hbuf), T, d_h, E, d_e, n,
                                static_cast<float*>(y), G, s);
         return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "fp32 forward launch");
     }
 
-    const bool fuse = L.C == 1;
-    static int clusters_cache[64];
-    static std::once_flag clusters_once[64];
-    int dev_id = 0;
-    cudaGetDevice(&dev_id);
-    int ncl = -1;
-    if (fuse && dev_id >= 0 && dev_id < 64) {
-        std::call_once(clusters_once[dev_id], [&]() { clusters_cache[dev_id] = decode_max_clusters(); });
-        ncl = clusters_cache[dev_id];
-        if (ncl > G / 4) ncl = G / 4;
-    }
-    if (fuse && ncl > 0 && 4 * ncl <= 160 && L.KB % 4 == 0 && E <= 256) {
+    if (L.path == Path::Decode) {
         // one chunk: clusters of 4 blocks, expert-in in k-half pairs, expert-out
         // row tiles summed inside the cluster (forward_decode.cu)
-        const int Gd = 4 * ncl;
+        const int Gd = decode_grid(L.C, d_h, E, G);
         CUtensorMap dmaps[5];
         if (!make_map_kpair(&dmaps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
             !make_map_kpair(&dmaps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
@@ -354,10 +403,13 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
             return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
         DcArgs da;
         da.gates = g;
+        da.counts_in = tables ? counts : nullptr;
+        da.idx_in = tables ? idx : nullptr;
+        da.tmask_in = tables ? tmask : nullptr;
         da.y = static_cast<__nv_bfloat16*>(y);
         da.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
         da.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
-        da.ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
+        da.ctl = ctl;
         da.T = T;
         da.d_h = d_h;
         da.E = E;
@@ -371,25 +423,31 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.trace = g_trace.load();
         da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1});
         // A cluster launch cannot also be cooperative; the grid is sized to the
-        // pairs that can be resident at once, and every wait is bounded.
+        // clusters that can be resident at once, and every wait is bounded.
         e = launch_forward_decode(da, dmaps, Gd, s);
         return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "single-chunk forward launch");
     }
-    if (!fuse) {
-        e = launch_chunk_union_plan(g, T, E, n, counts, idx, tmask, offsets, pair_ce, y, d_h, 2, s);
-        if (e != cudaSuccess) return cuda_fail(e, "union launch");
-    }
-    CUtensorMap maps[3];
+
+    // several chunks (or one the single-chunk kernel cannot take): group tables,
+    // then the group-major kernel (forward_group.cu)
+    int32_t* gcounts = reinterpret_cast<int32_t*>(ws + L.gcounts);
+    int32_t* goffsets = reinterpret_cast<int32_t*>(ws + L.goffsets);
+    int32_t* gpair = reinterpret_cast<int32_t*>(ws + L.gpair);
+    e = launch_group_plan(g, T, E, n, t_counts, t_idx, t_tmask, !tables, ctl, L.NG, L.NGr, gcounts, goffsets,
+                          gpair, static_cast<__nv_bfloat16*>(y), d_h, s);
+    if (e != cudaSuccess) return cuda_fail(e, "group plan launch");
+    CUtensorMap maps[4];
     if (!make_map(&maps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
         !make_map(&maps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
-        !make_map(&maps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128))
+        !make_map(&maps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
+        !make_map(&maps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)L.Pmax * L.N, (uint32_t)L.N))
         return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
-    TcArgs a;
+    GrArgs a;
     a.gates = g;
-    a.counts = counts;
-    a.offsets = offsets;
-    a.pair_ce = pair_ce;
-    a.tmask = tmask;
+    a.tmask = t_tmask;
+    a.gcounts = gcounts;
+    a.goffsets = goffsets;
+    a.gpair = gpair;
     a.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
     a.partA = reinterpret_cast<float*>(ws + L.partA);
     a.partB = reinterpret_cast<float*>(ws + L.partB);
@@ -397,8 +455,8 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
     a.cntB = reinterpret_cast<uint32_t*>(ws + L.cntB);
     a.cnt_a_len = L.Pmax * L.MT;
-    a.cnt_b_len = (long long)L.C * L.RT;
-    a.ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
+    a.cnt_b_len = (long long)L.NGr * L.RT;
+    a.ctl = ctl;
     a.y = static_cast<__nv_bfloat16*>(y);
     a.T = T;
     a.d_h = d_h;
@@ -406,18 +464,18 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.d_e = d_e;
     a.n = n;
     a.N = L.N;
-    a.C = L.C;
+    a.NT = L.NT;
+    a.NGr = L.NGr;
     a.KB = L.KB;
     a.MT = L.MT;
     a.RT = L.RT;
     a.KBe = L.KBe;
-    a.fuse_union = fuse ? 1 : 0;
-    a.wait_ns = g_wait_ns.load();
     a.skip_flag_unit = g_skip_flag.load();
-    a.trace = g_trace.load();
+    a.wait_ns = g_wait_ns.load();
     a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2});
-    e = launch_forward_tc(a, maps, G, s);
-    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "tensor-core forward launch");
+    a.trace = g_trace.load();
+    e = launch_forward_group(a, maps, G, s);
+    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "group forward launch");
 }
 
 // ------------------------------------------------------------------------
@@ -466,14 +524,9 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return fail(BLOCKFFN_ERR_CUDA, "no current CUDA device");
     const int G = num_sms_current();
-    static int clusters_cache[64];
-    static std::once_flag clusters_once[64];
-    std::call_once(clusters_once[dev], [&]() { clusters_cache[dev] = decode_max_clusters(); });
-    int ncl = clusters_cache[dev];
-    if (ncl > G / 4) ncl = G / 4;
-    if (ncl <= 0 || 4 * ncl > 160 || (d_h / 64) % 4 != 0 || E > 256)
+    const int Gd = decode_grid(1, d_h, E, G);
+    if (Gd <= 0)
         return fail(BLOCKFFN_ERR_UNSUPPORTED, "no-allocation forward: single-chunk kernel unavailable here");
-    const int Gd = 4 * ncl;
     const int N = n <= 16 ? 16 : 32;
     const int RT = d_h / 128;
     // scratch layout: control block and readiness counters (the part that must
@@ -502,6 +555,9 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
         return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     DcArgs da;
     da.gates = gates;
+    da.counts_in = nullptr;
+    da.idx_in = nullptr;
+    da.tmask_in = nullptr;
     da.y = static_cast<__nv_bfloat16*>(y);
     da.hbuf = reinterpret_cast<__nv_bfloat16*>(scratch + off_h);
     da.readyA = reinterpret_cast<uint32_t*>(scratch + off_ready);

@@ -32,6 +32,7 @@ enum : int32_t {
     kWaitMmaDone = 8,    // teardown waiting for the last MMAs
     kWaitPeers = 9,      // a split unit's block waiting for the other contributors
     kShapeKey = 10,      // (workspace error) bound to other shapes or another gating mode
+    kUnionTables = 11,   // (invalid argument) caller's counts / idx disagree with its token masks
 };
 
 // Control block at offset 0 of every forward workspace (256 bytes reserved).

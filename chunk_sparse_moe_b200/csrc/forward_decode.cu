@@ -91,9 +91,13 @@ struct RsShared {
     uint64_t a_pub;               // 1 arrival: this block's expert-in results are published
     uint32_t tmem_base;
     volatile int abort;
+    int abort0;                   // abort as thread 0 set it before the first block barrier
+    int tab_bad;                  // the caller's union tables disagree with their token masks
+    int ep_okA[2];                // epilogue: the two waits of an expert-in unit
+    int ep_okB[2];                // epilogue: the two waits of an expert-out row tile
+    int b_go, b_fail;             // epilogue: expert-out work may start / a summing warp gave up
     uint32_t epoch;
     int P;
-    int ep_ok;
     uint32_t trace_once;          // trace slots already stamped (first occurrence only)
     int pendA[2], pendB;          // parity of a receive phase armed but not seen complete, or -1
     float s_gate[2][32];          // gates of the current expert-in unit's expert, per token
@@ -287,20 +291,27 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const bool key_ok = key0 == 0ull || key0 == a.shape_key;
         if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
         sh.abort = st0 != 0 || !key_ok;
+        sh.abort0 = st0 != 0 || !key_ok;
     }
     if (warp >= 3) {
-        // the chunk's union, ascending (warps 3-6 take 32-expert groups; all of a
-        // lane's gate loads are issued before their first use)
+        // the chunk's union, ascending (warps 3-6 take 32-expert groups): from the
+        // gates (all of a lane's gate loads are issued before their first use), or
+        // from the caller's token masks
         const int ngroups = (a.E + 31) / 32;
+        const uint32_t live = nt >= 32 ? 0xffffffffu : ((1u << nt) - 1u);
         for (int g = warp - 3; g < ngroups; g += 4) {
             const int e = g * 32 + lane;
             const int ec = min(e, a.E - 1);
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __ldg(a.gates + (size_t)min(j, nt - 1) * a.E + ec);
             uint32_t bits = 0u;
+            if (a.tmask_in != nullptr) {
+                bits = e < a.E ? (__ldg(a.tmask_in + e) & live) : 0u;
+            } else {
+                float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) bits |= ((e < a.E && j < nt && v[j] != 0.f) ? 1u : 0u) << j;
+                for (int j = 0; j < 32; ++j) v[j] = __ldg(a.gates + (size_t)min(j, nt - 1) * a.E + ec);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) bits |= ((e < a.E && j < nt && v[j] != 0.f) ? 1u : 0u) << j;
+            }
             if (e < a.E) sh.s_tmask[e] = bits;
             const uint32_t bal = __ballot_sync(0xffffffffu, bits != 0u);
             if (lane == 0) sh.s_bal[g] = bal;
@@ -308,17 +319,43 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         named_bar_sync(1, 128);
         if (warp == 3) {
             int base = 0;
+            bool bad = false;
             for (int g = 0; g < ngroups; ++g) {
                 const uint32_t bal = sh.s_bal[g];
-                if ((bal >> lane) & 1u) sh.s_pair_e[base + __popc(bal & ((1u << lane) - 1u))] = g * 32 + lane;
+                const int slot = base + __popc(bal & ((1u << lane) - 1u));
+                if ((bal >> lane) & 1u) {
+                    sh.s_pair_e[slot] = g * 32 + lane;
+                    // the caller's index list must name the same experts in the same order
+                    if (a.idx_in != nullptr && __ldg(a.idx_in + slot) != g * 32 + lane) bad = true;
+                }
                 base += __popc(bal);
             }
-            if (lane == 0) sh.P = base;
+            if (a.idx_in != nullptr) {
+                for (int s2 = base + lane; s2 < a.E; s2 += 32)
+                    if (__ldg(a.idx_in + s2) != -1) bad = true;
+                if (lane == 0 && __ldg(a.counts_in) != base) bad = true;
+            }
+            bad = __any_sync(0xffffffffu, bad);
+            if (lane == 0) {
+                sh.P = base;
+                sh.tab_bad = bad ? 1 : 0;
+                if (bad) record_error(a.ctl, kErrInvalidArg, kUnionTables);
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (sh.tab_bad) {
+        // refused tables: nothing is computed (a uniform branch, so every thread
+        // takes the second barrier)
+        if (threadIdx.x == 0) sh.abort = 1;
+        __syncthreads();
+    }
+    // Whether this launch computes at all, the same in every thread: both words
+    // were written before the barrier above and are not written again.  (The
+    // volatile abort flag itself may be raised by any role at any time.)
+    const bool abort_at_start = sh.abort0 != 0 || sh.tab_bad != 0;
     const int P = sh.P;
     const RsWork wk = rs_work(G, P, MT, KPe, a.RT);
     const int nBt = wk.bHi - wk.bLo;                 // expert-out tiles per owned row tile
@@ -579,7 +616,11 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             const int oth = par ^ 1;
             for (int k2 = (int)blockIdx.x * 128 + et; k2 < a.E; k2 += G * 128) a.readyA[(size_t)oth * a.E + k2] = 0u;
         }
-        bool failed = sh.abort != 0;
+        // Every decision below that ends a loop is taken from shared memory after a
+        // named barrier (or, like this one, from values fixed before the block's
+        // first barrier), so the four epilogue warps always take the same path and
+        // meet the same named barriers.
+        bool failed = abort_at_start;
         if (P == 0 && blockIdx.x == 0 && !failed) {
             // empty union: y is all zeros
             for (size_t k2 = et; k2 < (size_t)nt * a.d_h; k2 += 128) a.y[k2] = __float2bfloat16_rn(0.f);
@@ -608,10 +649,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 if (ok && ua >= 2)
                     ok = wait_bar_cluster(&sh.freeA[b], (uint32_t)(((ua - 2) >> 1) & 1), limit_peer, &sh.abort,
                                           a.ctl, kWaitPeers) ? 1 : 0;
-                sh.ep_ok = ok;
+                sh.ep_okA[0] = ok;
             }
             named_bar_sync(1, 128);
-            if (!sh.ep_ok) { failed = true; break; }
+            if (!sh.ep_okA[0]) { failed = true; break; }
             tc_fence_after();
             uint32_t r[32];
             const uint32_t taddr = tmem + ((uint32_t)(qd * 32) << 16) + accA_col + (uint32_t)(b * N);
@@ -639,13 +680,13 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             if (et == 0) RS_TRACE_ONCE(kRtASent);
             const uint32_t bits = sh.s_tmask[e] >> tg;   // this half's token bits
             if (et == 0) {
-                sh.ep_ok = wait_bar_cluster(&sh.recvA[b], (uint32_t)((ua >> 1) & 1), limit_peer, &sh.abort, a.ctl,
-                                            kWaitPeers) ? 1 : 0;
-                if (sh.ep_ok) sh.pendA[b] = -1;
+                sh.ep_okA[1] = wait_bar_cluster(&sh.recvA[b], (uint32_t)((ua >> 1) & 1), limit_peer, &sh.abort,
+                                                a.ctl, kWaitPeers) ? 1 : 0;
+                if (sh.ep_okA[1]) sh.pendA[b] = -1;
                 RS_TRACE_ONCE(kRtAReady);
             }
             named_bar_sync(1, 128);
-            if (!sh.ep_ok) { failed = true; break; }
+            if (!sh.ep_okA[1]) { failed = true; break; }
             // h = (k-half 0) + (k-half 1): two terms, and the sum does not depend on
             // which block of the pair forms it
             float z[NH];
@@ -700,7 +741,14 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             if (wk.nA > 0) mbar_arrive(&sh.a_pub);   // the producer may load expert-out tiles now
         }
         // ---- expert-out row tiles: the cluster's 4 partials meet in shared memory
-        failed = failed || sh.abort;
+        // (failed is the same in the four warps here; the abort flag is read once,
+        // by one thread, and shared)
+        if (et == 0) {
+            sh.b_go = (!failed && !sh.abort) ? 1 : 0;
+            sh.b_fail = 0;
+        }
+        named_bar_sync(1, 128);
+        failed = failed || !sh.b_go;
         if (doB) {
             const uint32_t recv_u32 = smem_u32(recv);
             for (int k = 0; k < wk.nRT && !failed; ++k) {
@@ -709,10 +757,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 uint32_t r[32];
                 if (nBt > 0) {
                     if (et == 0)
-                        sh.ep_ok = wait_bar(&sh.accB_full[ab], (uint32_t)((k >> 1) & 1), limit, &sh.abort, a.ctl,
+                        sh.ep_okB[0] = wait_bar(&sh.accB_full[ab], (uint32_t)((k >> 1) & 1), limit, &sh.abort, a.ctl,
                                             kWaitAccFull) ? 1 : 0;
                     named_bar_sync(1, 128);
-                    if (!sh.ep_ok) { failed = true; break; }
+                    if (!sh.ep_okB[0]) { failed = true; break; }
                     tc_fence_after();
                     const uint32_t taddr = tmem + ((uint32_t)(qd * 32) << 16) + accB_col + (uint32_t)(ab * N);
                     if constexpr (N == 32) tmem_ld_32x32b_x32(taddr, r);
@@ -729,10 +777,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     // the receive area is reused: every other rank has summed the
                     // quadrants this block sent it for the previous row tile
                     if (et == 0)
-                        sh.ep_ok = wait_bar_cluster(&sh.freeB, (uint32_t)((k - 1) & 1), limit_peer, &sh.abort,
+                        sh.ep_okB[1] = wait_bar_cluster(&sh.freeB, (uint32_t)((k - 1) & 1), limit_peer, &sh.abort,
                                                     a.ctl, kWaitPeers) ? 1 : 0;
                     named_bar_sync(1, 128);
-                    if (!sh.ep_ok) { failed = true; break; }
+                    if (!sh.ep_okB[1]) { failed = true; break; }
                 }
                 if (qd != wk.cr) {
                     // rows of quadrant qd are summed by rank qd: slot cr of its receive
@@ -791,14 +839,15 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                             bulk_commit_group();
                             RS_TRACE_ONCE(kRtBReduced);
                         }
-                    } else {
-                        failed = true;
+                    } else if (lane == 0) {
+                        sh.b_fail = 1;   // the other warps learn it after the barrier below
                     }
                 }
                 if (k + 1 < wk.nRT) {
                     // hand the receive area back: re-arm it for the next row tile and
                     // tell the other ranks this block has summed what they sent
                     named_bar_sync(1, 128);
+                    failed = failed || sh.b_fail != 0;
                     if (et == 0 && !failed && !sh.abort) {
                         mbar_arrive_expect_tx(&sh.recvB, 3u * 32u * N * 4u);
                         sh.pendB = (k + 1) & 1;

@@ -31,8 +31,9 @@ constexpr int kF32Threads = 256;   // 8 warps x 8 rows
 __global__ void __launch_bounds__(kF32Threads) expert_in_f32_kernel(
     const float* __restrict__ x, const float* __restrict__ gates, const float* __restrict__ W_in,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ pair_ce,
-    const uint32_t* __restrict__ tmask, int T, int d_h, int E, int d_e, int n, int C,
+    const uint32_t* __restrict__ tmask, const Ctl* ctl, int T, int d_h, int E, int d_e, int n, int C,
     float* __restrict__ hbuf) {
+    if (__ldcg(&ctl->status) != 0) return;   // the union tables were refused (or an earlier error)
     __shared__ float sw[kF32Tile][kF32Tile + 1];   // [row][k]
     __shared__ float sx[32][kF32Tile + 1];         // [token][k]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,7 +86,8 @@ __global__ void __launch_bounds__(kF32Threads) expert_in_f32_kernel(
 __global__ void __launch_bounds__(kF32Threads) expert_out_f32_kernel(
     const float* __restrict__ W_out, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ pair_ce,
-    const float* __restrict__ hbuf, int T, int d_h, int d_e, int n, float* __restrict__ y) {
+    const float* __restrict__ hbuf, const Ctl* ctl, int T, int d_h, int d_e, int n, float* __restrict__ y) {
+    if (__ldcg(&ctl->status) != 0) return;
     __shared__ float sw[kF32Tile][kF32Tile + 1];   // [row i][q]
     __shared__ float sh[32][kF32Tile + 1];         // [token][q]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -130,21 +132,21 @@ __global__ void __launch_bounds__(kF32Threads) expert_out_f32_kernel(
 
 cudaError_t launch_forward_f32(const float* x, const float* gates, const float* W_in,
                                const float* W_out, const int32_t* counts, const int32_t* offsets,
-                               const int32_t* pair_ce, const uint32_t* tmask, float* hbuf,
-                               int T, int d_h, int E, int d_e, int n, float* y, int num_sms,
-                               cudaStream_t s) {
+                               const int32_t* pair_ce, const uint32_t* tmask, const Ctl* ctl,
+                               float* hbuf, int T, int d_h, int E, int d_e, int n, float* y,
+                               int num_sms, cudaStream_t s) {
     const int C = (T + n - 1) / n;
     if (C == 0) return cudaSuccess;
     if (C > 65535) return cudaErrorInvalidValue;
     const long long pmax = (long long)C * E;
     const int gridA = (int)(pmax < 8LL * num_sms ? pmax : 8LL * num_sms);
-    expert_in_f32_kernel<<<gridA, kF32Threads, 0, s>>>(x, gates, W_in, offsets, pair_ce, tmask, T, d_h,
+    expert_in_f32_kernel<<<gridA, kF32Threads, 0, s>>>(x, gates, W_in, offsets, pair_ce, tmask, ctl, T, d_h,
                                                        E, d_e, n, C, hbuf);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     dim3 gridB((d_h + kF32Tile - 1) / kF32Tile, C);
-    expert_out_f32_kernel<<<gridB, kF32Threads, 0, s>>>(W_out, counts, offsets, pair_ce, hbuf, T, d_h,
-                                                        d_e, n, y);
+    expert_out_f32_kernel<<<gridB, kF32Threads, 0, s>>>(W_out, counts, offsets, pair_ce, hbuf, ctl, T,
+                                                        d_h, d_e, n, y);
     return cudaGetLastError();
 }
 

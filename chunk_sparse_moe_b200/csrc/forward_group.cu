@@ -1,0 +1,749 @@
+// forward_group.cu -- the multi-chunk union-expert forward on the sm_100a tensor
+// cores (bf16 in, fp32 accumulation in TMEM), expert-major over groups of chunks.
+//
+// Pages: "BlockFFN: Sparse Mixture-of-Experts Optimized for End-Device
+// Deployment", Core Concept (for n tokens at once only the union of their
+// activated experts is computed; unneeded activations are masked after
+// computing) and Architecture Overview (non-gated Swish experts, d_e << d_h);
+// the layer sums gate * expert output over the experts (Full BlockFFN Layer with
+// Combined Losses).
+//
+// Groups.  The chunks are taken NG at a time: a group is NT = NG * n consecutive
+// tokens (NT <= N, the MMA's token count, 128 or 256) made of whole chunks.  The
+// group's expert set is the union of its chunks' unions, ascending; each expert
+// of it runs once over all NT tokens, and every token's own mask selects its
+// activations afterwards.  A token whose gate is zero contributes an exact zero,
+// so the result is the per-chunk union-then-mask result; each weight tile is
+// read once per group instead of once per chunk, and every MMA is 128 x N x 16.
+//
+// Work.  For every group G and expert e of its set (a "pair" p):
+//   expert-in  : h^T[d_e, N]  = W_in_e[d_e, d_h] . x_G^T[d_h, N]           (A units)
+//                h'[j, :]     = bit_j ? g[t_j, e] * Swish(h[j, :]) : 0      (epilogue)
+//   expert-out : y_G^T[d_h,N] = sum_{e in U_G, ascending} W_out_e . h'_e^T  (B units)
+// bit_j is token t_j's bit in its chunk's token mask (the chunk union tables).
+//
+// Schedule.  One persistent block per SM (cooperative launch: all resident).  The
+// A work (pairs x 128-row tiles x 64-wide k-blocks) and the B work (groups x
+// 128-row tiles of y x (expert, k-block)) are each cut into equal contiguous
+// ranges of 16 KB weight tiles, one range of each per block, so every SM streams
+// the same number of weight bytes and A tiles come before B tiles everywhere.  A
+// unit split across blocks is finished by each contributor for its share of the
+// rows, summing the partials in block order (a fixed order: results do not depend
+// on timing).  An expert-out tile waits, with a bounded spin, until every
+// contributor of the expert-in unit it reads has written its rows of h'.
+//
+// Roles (224 threads): warp 0 issues the weight/activation TMA loads, warp 1
+// issues the MMAs (the whole warp runs the loop, one elected lane issues), warp 2
+// owns TMEM and loads h' tiles by TMA once their flag is set, warps 3-6 drain the
+// accumulators (TMEM -> registers, 32 columns at a time) and do the split
+// reductions, Swish, gate, mask and stores.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace bffn {
+
+namespace {
+
+constexpr int kGrThreads = 224;
+constexpr int kGrWBytes = 128 * 128;            // weight tile: 128 rows x 64 bf16
+constexpr int kGrMaxE = 256;
+constexpr int kGrMaxContrib = 160;              // >= blocks per launch (one per SM)
+constexpr int kGrSmemBudget = 200 * 1024;       // pipeline stages
+
+template <int N>
+struct GrCfg {
+    static constexpr int kActBytes = N * 128;   // activation tile: N rows x 64 bf16
+    static constexpr int kStageBytes = kGrWBytes + kActBytes;
+    static constexpr int kStages = kGrSmemBudget / kStageBytes;
+    static constexpr int kTmemCols = 2 * N;     // two accumulators of N columns
+};
+
+template <int N>
+struct GrShared {
+    uint64_t full_w[GrCfg<N>::kStages];    // weight (+x) tile landed
+    uint64_t full_h[GrCfg<N>::kStages];    // h' tile landed (B) or nothing to load (A)
+    uint64_t empty[GrCfg<N>::kStages];     // MMAs reading the stage are done
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    volatile int abort;
+    int abort0;                            // abort as set before the first block barrier
+    uint32_t epoch;
+    int ep_wait[2];
+    int ep_ok;
+    int s_contrib[kGrMaxContrib];
+    int32_t s_elist[kGrMaxE];              // producer: experts of the current B unit
+    float s_gv[N];                         // epilogue: the unit's gates (0 where masked)
+    uint32_t s_bits[N / 32];               // epilogue: the unit's token bits
+};
+
+struct GrSeg {
+    int kind;                  // 0: expert-in (A), 1: expert-out (B)
+    long long lo, hi;          // this block's tiles of the unit, [lo, hi)
+    long long first, last;     // all tiles of the unit, [first, last]
+    int g, e, p, mt;           // A: group, expert, pair, row tile of W_in_e
+    int rt, cnt, off;          // B: row tile of y, the group's union size and first pair
+    uint32_t unit;
+};
+
+__device__ __forceinline__ long long gr_range_lo(long long total, int G, int i) {
+    if (total < (1LL << 31) / (G + 1)) return (long long)((uint32_t)total * (uint32_t)i / (uint32_t)G);
+    return total * i / G;
+}
+__device__ __forceinline__ int gr_block_of(long long j, long long total, int G) {
+    if (total < (1LL << 31) / (G + 1)) return (int)((((uint32_t)j + 1u) * (uint32_t)G - 1u) / (uint32_t)total);
+    return (int)(((j + 1) * G - 1) / total);
+}
+
+// The blocks holding tiles of a unit spanning tiles [first, last]: q0..q1 with a
+// non-empty range; n of them, and the rank of `me` among them (-1 if none).
+struct GrContrib {
+    int q0, q1, n, rank;
+};
+__device__ __forceinline__ GrContrib gr_contributors(long long first, long long last, long long total, int G,
+                                                     int me) {
+    GrContrib c;
+    c.q0 = gr_block_of(first, total, G);
+    c.q1 = gr_block_of(last, total, G);
+    if (total >= G) {
+        c.n = c.q1 - c.q0 + 1;
+        c.rank = (me >= c.q0 && me <= c.q1) ? me - c.q0 : -1;
+        return c;
+    }
+    c.n = 0;
+    c.rank = -1;
+    for (int qq = c.q0; qq <= c.q1; ++qq) {
+        if (gr_range_lo(total, G, qq + 1) > gr_range_lo(total, G, qq)) {
+            if (qq == me) c.rank = c.n;
+            ++c.n;
+        }
+    }
+    return c;
+}
+
+struct GrIter {
+    long long aLo, aHi, bLo, bHi, cur;
+    int phase;
+    __device__ void init(long long a0, long long a1, long long b0, long long b1) {
+        aLo = a0; aHi = a1; bLo = b0; bHi = b1; cur = a0; phase = 0;
+    }
+    __device__ bool next(const GrArgs& a, GrSeg& s) {
+        if (phase == 0) {
+            if (cur < aHi) {
+                const long long u = cur / a.KB;
+                s.kind = 0;
+                s.p = (int)(u / a.MT);
+                s.mt = (int)(u % a.MT);
+                const int ge = a.gpair[s.p];
+                s.g = ge >> 8;
+                s.e = ge & 255;
+                s.first = u * a.KB;
+                s.last = s.first + a.KB - 1;
+                s.unit = (uint32_t)u;
+                s.lo = cur;
+                s.hi = min(aHi, s.last + 1);
+                cur = s.hi;
+                return true;
+            }
+            phase = 1;
+            cur = bLo;
+        }
+        if (phase == 1) {
+            if (cur < bHi) {
+                const long long per_pair = (long long)a.RT * a.KBe;
+                const int q = (int)(cur / per_pair);
+                const int g = a.gpair[q] >> 8;
+                const int off = a.goffsets[g];
+                const int cnt = a.gcounts[g];
+                const long long base = (long long)off * per_pair;
+                const long long unit_tiles = (long long)cnt * a.KBe;
+                const int rt = (int)((cur - base) / unit_tiles);
+                s.kind = 1;
+                s.g = g;
+                s.off = off;
+                s.cnt = cnt;
+                s.rt = rt;
+                s.first = base + rt * unit_tiles;
+                s.last = s.first + unit_tiles - 1;
+                s.unit = (uint32_t)(g * a.RT + rt);
+                s.lo = cur;
+                s.hi = min(bHi, s.last + 1);
+                cur = s.hi;
+                return true;
+            }
+            phase = 2;
+        }
+        return false;
+    }
+};
+
+__device__ __forceinline__ float gr_swish(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// Timeline stamps (globaltimer, ns) of one launch, written only when a trace
+// buffer is attached: per block 64 slots.
+enum : int {
+    kGtStart = 0, kGtPrologue = 1, kGtFirstLoad = 2, kGtLastALoad = 3, kGtLastACommit = 4,
+    kGtAFlushed = 5, kGtFirstFlag = 6, kGtLastBCommit = 7, kGtEpiEnd = 8, kGtEnd = 9,
+    kGtFirstAcc = 10, kGtFirstBLoad = 11, kGtLastLoad = 12, kGtSlots = 64
+};
+#define GR_TRACE(slot) \
+    do { if (a.trace) a.trace[(size_t)blockIdx.x * kGtSlots + (slot)] = globaltimer_ns(); } while (0)
+
+}  // namespace
+
+template <int N>
+__global__ void __launch_bounds__(kGrThreads, 1)
+union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_win,
+                   const __grid_constant__ CUtensorMap tm_wout, const __grid_constant__ CUtensorMap tm_h,
+                   const GrArgs a) {
+    using Cfg = GrCfg<N>;
+    constexpr int kStages = Cfg::kStages;
+    constexpr int kStageBytes = Cfg::kStageBytes;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    GrShared<N>& sh = *reinterpret_cast<GrShared<N>*>(smem + kStages * kStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, cta = blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        GR_TRACE(kGtStart);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sh.full_w[s], 1);
+            mbar_init(&sh.full_h[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sh.acc_full[s], 1);
+            mbar_init(&sh.acc_empty[s], 4);
+        }
+        mbar_init(&sh.mma_done, 1);
+        fence_mbar_init();
+        // written by earlier launches only: plain L2 loads
+        const int32_t st0 = __ldcg(&a.ctl->status);
+        const uint32_t ep0 = __ldcg(&a.ctl->epoch);
+        const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
+        const bool key_ok = key0 == 0ull || key0 == a.shape_key;
+        if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
+        sh.abort = st0 != 0 || !key_ok;
+        sh.abort0 = st0 != 0 || !key_ok;
+        sh.epoch = ep0;
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_win);
+        prefetch_tmap(&tm_wout);
+        prefetch_tmap(&tm_h);
+    }
+    if (warp == 2) {
+        tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) GR_TRACE(kGtPrologue);
+
+    const uint32_t tmem = sh.tmem_base;
+    const int P = a.goffsets[a.NGr];
+    const uint32_t stamp = sh.epoch + 1u;
+    const int par = (int)(sh.epoch & 1u);
+    uint32_t* const cntA = a.cntA + (size_t)par * a.cnt_a_len;
+    uint32_t* const readyA = a.readyA + (size_t)par * a.cnt_a_len;
+    uint32_t* const cntB = a.cntB + (size_t)par * a.cnt_b_len;
+    const long long NA = (long long)P * a.MT * a.KB;
+    const long long NB = (long long)P * a.RT * a.KBe;
+    const long long aLo = NA > 0 ? gr_range_lo(NA, G, cta) : 0, aHi = NA > 0 ? gr_range_lo(NA, G, cta + 1) : 0;
+    const long long bLo = NB > 0 ? gr_range_lo(NB, G, cta) : 0, bHi = NB > 0 ? gr_range_lo(NB, G, cta + 1) : 0;
+    // waits on other blocks run out after wait_ns; waits on this block's own
+    // pipeline are downstream of those and get twice as long, so the first
+    // timeout recorded names the root cause
+    const uint64_t limit_peer = a.wait_ns;
+    const uint64_t limit = 2 * a.wait_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer --
+        // A group's x tile is read once per expert of its set: kept in L2.  Weight
+        // tiles are read once per group that uses the expert, by blocks that run at
+        // about the same time: the normal policy.
+        const uint64_t pol_weights = policy_evict_normal();
+        const uint64_t pol_keep = policy_evict_last();
+        GrIter it;
+        it.init(aLo, aHi, bLo, bHi);
+        GrSeg sg;
+        long long i = 0;
+        int st = 0;
+        uint32_t ph = 0u;
+        bool stop = sh.abort0 != 0;   // the same in all 32 lanes
+        while (!stop && it.next(a, sg)) {
+            if (sg.kind == 1) {
+                for (int k = lane; k < sg.cnt; k += 32) sh.s_elist[k] = a.gpair[sg.off + k] & 255;
+                __syncwarp();
+            }
+            if (lane == 0) {
+                int sidx = 0, kb = 0;
+                if (sg.kind == 1) {
+                    const long long local = sg.lo - sg.first;
+                    sidx = (int)(local / a.KBe);
+                    kb = (int)(local - (long long)sidx * a.KBe);
+                }
+                for (long long j = sg.lo; j < sg.hi; ++j, ++i) {
+                    if (!wait_bar(&sh.empty[st], ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t* w = smem + st * kStageBytes;
+                    if (i == 0) GR_TRACE(kGtFirstLoad);
+                    if (sg.kind == 0) {
+                        GR_TRACE(kGtLastALoad);
+                        const int kbA = (int)(j - sg.first);
+                        mbar_arrive_expect_tx(&sh.full_w[st], kGrWBytes + Cfg::kActBytes);
+                        tma_load_2d(w, &tm_win, &sh.full_w[st], kbA * 64, sg.e * a.d_e + sg.mt * 128, pol_weights);
+                        tma_load_2d(w + kGrWBytes, &tm_x, &sh.full_w[st], kbA * 64, sg.g * a.NT, pol_keep);
+                    } else {
+                        const int e = sh.s_elist[sidx];
+                        mbar_arrive_expect_tx(&sh.full_w[st], kGrWBytes);
+                        tma_load_2d(w, &tm_wout, &sh.full_w[st], kb * 64, e * a.d_h + sg.rt * 128, pol_weights);
+                        if (++kb == a.KBe) {
+                            kb = 0;
+                            ++sidx;
+                        }
+                    }
+                    if (++st == kStages) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+            i = __shfl_sync(0xffffffffu, i, 0);
+            st = __shfl_sync(0xffffffffu, st, 0);
+            ph = __shfl_sync(0xffffffffu, ph, 0);
+            __syncwarp();
+        }
+        if (lane == 0) {
+            GR_TRACE(kGtLastLoad);
+            // let every issued copy land before the block can exit
+            for (long long k = i - kStages < 0 ? 0 : i - kStages; k < i; ++k)
+                wait_bar_drain(&sh.full_w[k % kStages], (uint32_t)((k / kStages) & 1), limit, a.ctl);
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer --
+        const bool leader = elect_one();
+        const uint32_t idesc = idesc_bf16_f32(128, N);
+        const uint64_t desc0 = sw128_kmajor_desc(smem_u32(smem));
+        GrIter it;
+        it.init(aLo, aHi, bLo, bHi);
+        GrSeg sg;
+        int st = 0;
+        uint32_t ph = 0u;
+        uint32_t rw = 0u, rh = 0u;   // the current stage's barriers as last tested
+        uint32_t acc_i = 0;
+        bool stop = __shfl_sync(0xffffffffu, sh.abort, 0) != 0;
+        while (!stop && it.next(a, sg)) {
+            const int ab = (int)(acc_i & 1u);
+            const uint32_t aph = (acc_i >> 1) & 1u;
+            if (!wait_bar_warp(&sh.acc_empty[ab], aph ^ 1u, limit, &sh.abort, a.ctl, kWaitAccEmpty)) break;
+            tc_fence_after();
+            const uint32_t d = tmem + (uint32_t)(ab * N);
+            for (long long j = sg.lo; j < sg.hi; ++j) {
+                if (!__all_sync(0xffffffffu, rw & rh) &&
+                    (!wait_bar_warp(&sh.full_w[st], ph, limit, &sh.abort, a.ctl, kWaitFullW) ||
+                     !wait_bar_warp(&sh.full_h[st], ph, limit, &sh.abort, a.ctl, kWaitFullH))) {
+                    stop = true;
+                    break;
+                }
+                tc_fence_after();
+                const int st_n = st + 1 == kStages ? 0 : st + 1;
+                const uint32_t ph_n = st + 1 == kStages ? ph ^ 1u : ph;
+                rw = mbar_test_wait(&sh.full_w[st_n], ph_n);
+                rh = mbar_test_wait(&sh.full_h[st_n], ph_n);
+                if (leader) {
+                    const uint64_t ds = desc0 + (uint64_t)(st * (kStageBytes >> 4));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(d, ds + (uint64_t)((kk * 32) >> 4), ds + (uint64_t)((kGrWBytes + kk * 32) >> 4),
+                                  idesc, (j > sg.lo || kk > 0) ? 1u : 0u);
+                    umma_commit(&sh.empty[st]);
+                }
+                __syncwarp();
+                st = st_n;
+                ph = ph_n;
+            }
+            if (stop) break;
+            if (leader) {
+                umma_commit(&sh.acc_full[ab]);
+                GR_TRACE(sg.kind == 0 ? kGtLastACommit : kGtLastBCommit);
+            }
+            __syncwarp();
+            ++acc_i;
+        }
+        if (leader) umma_commit(&sh.mma_done);
+        __syncwarp();
+    } else if (warp == 2) {
+        // ----------------------------------------------------- h' tile loader --
+        // An expert-in stage carries no h': lane 0 just arrives.  For an expert-out
+        // tile, lane 0 waits (bounded) until every contributor of the expert-in
+        // unit holding the tile's 64 columns of h' has written its rows, then moves
+        // the [N x 64] slice by TMA (it lands in the 128-byte-swizzled layout the
+        // MMA reads).
+        GrIter it;
+        it.init(aLo, aHi, bLo, bHi);
+        GrSeg sg;
+        int st = 0;
+        uint32_t ph = 0u;
+        long long i = 0, nB = 0;
+        bool stop = sh.abort != 0;
+        uint32_t last_u = 0xffffffffu;
+        const uint64_t pol = policy_evict_last();   // an h' tile is read once per row tile of y
+        if (lane == 0) {
+            while (!stop && it.next(a, sg)) {
+                int sidx = 0, kb = 0;
+                if (sg.kind == 1) {
+                    const long long local = sg.lo - sg.first;
+                    sidx = (int)(local / a.KBe);
+                    kb = (int)(local - (long long)sidx * a.KBe);
+                }
+                for (long long j = sg.lo; j < sg.hi; ++j, ++i) {
+                    if (!wait_bar(&sh.empty[st], ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
+                        stop = true;
+                        break;
+                    }
+                    if (sg.kind == 0) {
+                        mbar_arrive(&sh.full_h[st]);
+                    } else {
+                        const int p = sg.off + sidx;
+                        const uint32_t u = (uint32_t)(p * a.MT + (kb >> 1));
+                        if (u != last_u) {
+                            const long long fA = (long long)u * a.KB;
+                            const int ncA = gr_contributors(fA, fA + a.KB - 1, NA, G, -1).n;
+                            if (!wait_count(&readyA[u], (uint32_t)ncA, limit_peer, &sh.abort, a.ctl)) {
+                                stop = true;
+                                break;
+                            }
+                            if (nB == 0) GR_TRACE(kGtFirstFlag);
+                            // the h' stores were made visible to this thread by the
+                            // acquire; the async proxy reads them next
+                            fence_proxy_async_global();
+                            last_u = u;
+                        }
+                        mbar_arrive_expect_tx(&sh.full_h[st], (uint32_t)Cfg::kActBytes);
+                        tma_load_2d(smem + st * kStageBytes + kGrWBytes, &tm_h, &sh.full_h[st], kb * 64, p * N,
+                                    pol);
+                        ++nB;
+                        if (++kb == a.KBe) {
+                            kb = 0;
+                            ++sidx;
+                        }
+                    }
+                    if (++st == kStages) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // no copy into this block's shared memory outlives it: the last
+            // kStages stages issued (only B stages carry bytes)
+            if (nB > 0) {
+                for (long long k = i - kStages < 0 ? 0 : i - kStages; k < i; ++k)
+                    wait_bar_drain(&sh.full_h[k % kStages], (uint32_t)((k / kStages) & 1), limit, a.ctl);
+            }
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------------- epilogue (3-6) --
+        const int q = warp & 3;
+        const int row = q * 32 + lane;           // accumulator row = TMEM lane
+        const int et = threadIdx.x - 96;         // 0..127
+        {
+            // zero the other parity's counters: the launch before this one used
+            // them and has finished; the launch after this one will use them
+            const int oth = par ^ 1;
+            const long long step = (long long)G * 128;
+            for (long long k = (long long)cta * 128 + et; k < a.cnt_a_len; k += step) {
+                a.cntA[(size_t)oth * a.cnt_a_len + k] = 0u;
+                a.readyA[(size_t)oth * a.cnt_a_len + k] = 0u;
+            }
+            for (long long k = (long long)cta * 128 + et; k < a.cnt_b_len; k += step)
+                a.cntB[(size_t)oth * a.cnt_b_len + k] = 0u;
+        }
+        // the gates of expert e for the tokens of group g, zero where the token's
+        // bit in its chunk's mask is clear or the token lies past the group or T,
+        // and the bits themselves; staged in shared memory by the 128 threads
+        auto stage_gates = [&](int g, int e) {
+            for (int j = et; j < N; j += 128) {
+                const int t = g * a.NT + j;
+                bool bit = false;
+                float gv = 0.f;
+                if (j < a.NT && t < a.T) {
+                    const int c = t / a.n;
+                    bit = ((a.tmask[(size_t)c * a.E + e] >> (t - c * a.n)) & 1u) != 0u;
+                    gv = a.gates[(size_t)t * a.E + e];
+                }
+                sh.s_gv[j] = bit ? gv : 0.f;
+                const uint32_t bal = __ballot_sync(0xffffffffu, bit);
+                if (lane == 0) sh.s_bits[j >> 5] = bal;
+            }
+            named_bar_sync(1, 128);
+        };
+
+        GrSeg pend_sg[2];
+        GrContrib pend_cb[2];
+        int npend = 0;
+        // the same in every epilogue thread (fixed before the first barrier); later
+        // decisions come from shared words read after named barriers
+        bool failed = sh.abort0 != 0;   // (the tables are not read after an error)
+
+        // finish the rows [r0, r1) slice of split unit (sg, cb): sum the partials
+        // in block order, then gated Swish + mask into h' (A) or store y (B)
+        auto finish_split = [&](const GrSeg& sg, const GrContrib& cb) -> bool {
+            const long long total = sg.kind == 0 ? NA : NB;
+            uint32_t* cnt = (sg.kind == 0 ? cntA : cntB) + sg.unit;
+            if (et == 0) {
+                sh.ep_ok = wait_count(cnt, (uint32_t)cb.n, limit_peer, &sh.abort, a.ctl, kWaitPeers) ? 1 : 0;
+                int k = 0;
+                for (int qq = cb.q0; qq <= cb.q1 && k < kGrMaxContrib; ++qq) {
+                    const long long lo = gr_range_lo(total, G, qq);
+                    if (gr_range_lo(total, G, qq + 1) > lo) sh.s_contrib[k++] = qq * 2 + (lo >= sg.first ? 0 : 1);
+                }
+            }
+            named_bar_sync(1, 128);
+            if (!sh.ep_ok) return false;
+            if (sg.kind == 0) stage_gates(sg.g, sg.e);
+            const float* part = sg.kind == 0 ? a.partA : a.partB;
+            const float4* pbase = reinterpret_cast<const float4*>(part);
+            const int r0 = cb.rank * 128 / cb.n, r1 = (cb.rank + 1) * 128 / cb.n;
+            const int nrows = r1 - r0;
+            const int nvalid = min(a.NT, a.T - sg.g * a.NT);   // tokens of the group
+            // items (row, token quad) of the slice; per pass every contributor's
+            // float4 is requested before any is used, 8 contributors at a time
+            const int nitems = nrows * (N / 4);
+            for (int base = 0; base < nitems; base += 256) {
+                int rr[2], kq[2];
+                bool on[2];
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    const int itx = base + m * 128 + et;
+                    on[m] = itx < nitems;
+                    const int ic = on[m] ? itx : 0;
+                    rr[m] = r0 + ic % nrows;       // consecutive threads: consecutive rows
+                    kq[m] = ic / nrows;            // token quad
+                }
+                float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+                for (int c0 = 0; c0 < cb.n; c0 += 8) {
+                    float4 t4[2][8];
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            t4[m][u] = __ldcg(pbase + (size_t)sh.s_contrib[min(c0 + u, cb.n - 1)] * (N * 32) +
+                                              kq[m] * 128 + rr[m]);
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            if (c0 + u < cb.n) {
+                                acc[m].x += t4[m][u].x;
+                                acc[m].y += t4[m][u].y;
+                                acc[m].z += t4[m][u].z;
+                                acc[m].w += t4[m][u].w;
+                            }
+                        }
+                }
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    if (!on[m]) continue;
+                    const float z[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
+                    if (sg.kind == 0) {
+                        __nv_bfloat16* hrow = a.hbuf + (size_t)sg.p * N * a.d_e + sg.mt * 128 + rr[m];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int j = 4 * kq[m] + u;
+                            const bool bit = (sh.s_bits[j >> 5] >> (j & 31)) & 1u;
+                            const float h = bit ? sh.s_gv[j] * gr_swish(z[u]) : 0.f;
+                            hrow[(size_t)j * a.d_e] = __float2bfloat16_rn(h);
+                        }
+                    } else {
+                        __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + rr[m];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int j = 4 * kq[m] + u;
+                            if (j < nvalid) ycol[(size_t)j * a.d_h] = __float2bfloat16_rn(z[u]);
+                        }
+                    }
+                }
+            }
+            // every thread is done with sh.ep_ok and (A) the staged gates before the
+            // next unit's wait rewrites them
+            named_bar_sync(1, 128);
+            return true;
+        };
+        // this block's rows of h' for expert-in unit `unit` are written: count it in
+        auto announce_ready = [&](uint32_t unit) {
+            __threadfence();
+            named_bar_sync(1, 128);
+            if (et == 0 && (int)unit != a.skip_flag_unit) atomicAdd(&readyA[unit], 1u);
+        };
+        auto flush_pending = [&]() -> bool {
+            for (int k = 0; k < npend; ++k) {
+                if (!finish_split(pend_sg[k], pend_cb[k])) return false;
+                if (pend_sg[k].kind == 0) announce_ready(pend_sg[k].unit);
+            }
+            npend = 0;
+            return true;
+        };
+
+        GrIter it;
+        it.init(aLo, aHi, bLo, bHi);
+        GrSeg sg;
+        uint32_t acc_i = 0;
+        int cur_kind = 0;
+        while (!failed && it.next(a, sg)) {
+            if (sg.kind != cur_kind) {
+                if (!flush_pending()) { failed = true; break; }
+                cur_kind = sg.kind;
+                if (et == 0) GR_TRACE(kGtAFlushed);
+            }
+            const long long total = sg.kind == 0 ? NA : NB;
+            const GrContrib cb = gr_contributors(sg.first, sg.last, total, G, cta);
+            // stage this unit's gates while its accumulator completes
+            if (sg.kind == 0 && cb.n == 1) stage_gates(sg.g, sg.e);
+            const int ab = (int)(acc_i & 1u);
+            const uint32_t aph = (acc_i >> 1) & 1u;
+            // one thread waits and the 128 threads take its decision together, so
+            // the named barriers below always see all of them
+            if (et == 0)
+                sh.ep_wait[acc_i & 1u] =
+                    wait_bar(&sh.acc_full[ab], aph, limit, &sh.abort, a.ctl, kWaitAccFull) ? 1 : 0;
+            named_bar_sync(1, 128);
+            if (!sh.ep_wait[acc_i & 1u]) { failed = true; break; }
+            tc_fence_after();
+            if (et == 0 && acc_i == 0) GR_TRACE(kGtFirstAcc);
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * N);
+            const int nvalid = min(a.NT, a.T - sg.g * a.NT);   // tokens of the group
+            if (cb.n == 1) {
+                // the whole unit is here: all 128 rows straight from the accumulator
+                if (sg.kind == 0) {
+                    __nv_bfloat16* hrow = a.hbuf + (size_t)sg.p * N * a.d_e + sg.mt * 128 + row;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < N; c0 += 32) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
+                        tmem_ld_wait();
+                        const uint32_t bits = sh.s_bits[c0 >> 5];
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) {
+                            const float h = ((bits >> u) & 1u) ? sh.s_gv[c0 + u] * gr_swish(__uint_as_float(r[u])) : 0.f;
+                            hrow[(size_t)(c0 + u) * a.d_e] = __float2bfloat16_rn(h);
+                        }
+                    }
+                } else {
+                    __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + row;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < N; c0 += 32) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int u = 0; u < 32; ++u)
+                            if (c0 + u < nvalid) ycol[(size_t)(c0 + u) * a.d_h] = __float2bfloat16_rn(__uint_as_float(r[u]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.acc_empty[ab]);
+                ++acc_i;
+                if (sg.kind == 0) announce_ready(sg.unit);   // also frees the staged gates
+            } else {
+                // publish this block's partial tile and count it in; the slice is
+                // finished in the second pass.  Layout: float4 (token quad k, row)
+                // at k * 128 + row.
+                float* part = sg.kind == 0 ? a.partA : a.partB;
+                uint32_t* cnt = (sg.kind == 0 ? cntA : cntB) + sg.unit;
+                const long long myLo = sg.kind == 0 ? aLo : bLo;
+                const int myslot = myLo >= sg.first ? 0 : 1;
+                float4* dst = reinterpret_cast<float4*>(part + (size_t)(cta * 2 + myslot) * (N * 128)) + row;
+#pragma unroll 1
+                for (int c0 = 0; c0 < N; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        dst[(c0 / 4 + k) * 128] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                                                              __uint_as_float(r[4 * k + 2]),
+                                                              __uint_as_float(r[4 * k + 3]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.acc_empty[ab]);
+                ++acc_i;
+                __threadfence();
+                named_bar_sync(1, 128);
+                if (et == 0) atomicAdd(cnt, 1u);
+                if (npend < 2) {
+                    pend_sg[npend] = sg;
+                    pend_cb[npend] = cb;
+                    ++npend;
+                }
+            }
+        }
+        if (!failed) flush_pending();
+        if (et == 0) GR_TRACE(kGtEpiEnd);
+    }
+
+    // ------------------------------------------------------------ teardown --
+    __syncthreads();
+    if (warp == 2) {
+        if (lane == 0) wait_bar_drain(&sh.mma_done, 0, limit, a.ctl);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const uint32_t old = atomicAdd(&a.ctl->done, 1u);
+        if (old == (uint32_t)(G - 1)) {
+            a.ctl->done = 0u;
+            atomicExch(&a.ctl->epoch, stamp);
+        }
+        GR_TRACE(kGtEnd);
+    }
+}
+
+template <int N>
+static size_t group_smem_bytes() {
+    return 1024 + (size_t)GrCfg<N>::kStages * GrCfg<N>::kStageBytes + sizeof(GrShared<N>);
+}
+
+template <int N>
+static cudaError_t launch_group_n(const GrArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s) {
+    const size_t smem = group_smem_bytes<N>();
+    cudaError_t err =
+        cudaFuncSetAttribute(union_expert_group<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kGrThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, union_expert_group<N>, maps[0], maps[1], maps[2], maps[3], a);
+}
+
+cudaError_t launch_forward_group(const GrArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s) {
+    if (grid > kGrMaxContrib || a.E > kGrMaxE) return cudaErrorInvalidValue;
+    if (a.N == 256) return launch_group_n<256>(a, maps, grid, s);
+    if (a.N == 128) return launch_group_n<128>(a, maps, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace bffn

@@ -26,50 +26,55 @@ cudaError_t launch_residual_layernorm(const void* y, const void* x, const float*
 cudaError_t launch_chunk_union(const float* gates, int T, int E, int n, int32_t* counts,
                                int32_t* idx, uint32_t* tmask, cudaStream_t s);
 
+// compute_union: tables from the gates; otherwise the caller's tables are checked
+// (a mismatch records an error in ctl and the forward computes nothing)
 cudaError_t launch_chunk_union_plan(const float* gates, int T, int E, int n, int32_t* counts,
-                                    int32_t* idx, uint32_t* tmask, int32_t* offsets,
-                                    int32_t* pair_ce, void* y, int d_h, int y_elem_bytes,
-                                    cudaStream_t s);
+                                    int32_t* idx, uint32_t* tmask, bool compute_union, Ctl* ctl,
+                                    int32_t* offsets, int32_t* pair_ce, void* y, int d_h,
+                                    int y_elem_bytes, cudaStream_t s);
+
+// group tables of the multi-chunk forward (see union.cu)
+cudaError_t launch_group_plan(const float* gates, int T, int E, int n, int32_t* counts, int32_t* idx,
+                              uint32_t* tmask, bool compute_union, Ctl* ctl, int NG, int NGr,
+                              int32_t* gcounts, int32_t* goffsets, int32_t* gpair, __nv_bfloat16* y,
+                              int d_h, cudaStream_t s);
 
 cudaError_t launch_forward_f32(const float* x, const float* gates, const float* W_in,
                                const float* W_out, const int32_t* counts, const int32_t* offsets,
-                               const int32_t* pair_ce, const uint32_t* tmask, float* hbuf,
-                               int T, int d_h, int E, int d_e, int n, float* y, int num_sms,
-                               cudaStream_t s);
+                               const int32_t* pair_ce, const uint32_t* tmask, const Ctl* ctl,
+                               float* hbuf, int T, int d_h, int E, int d_e, int n, float* y,
+                               int num_sms, cudaStream_t s);
 
-// Arguments of the tensor-core union-expert forward (bf16).
-struct TcArgs {
+// Arguments of the multi-chunk group forward (forward_group.cu).
+struct GrArgs {
     const float* gates;       // [T, E]
-    const int32_t* counts;    // [C]       (plan tables; unused when fuse_union)
-    const int32_t* offsets;   // [C + 1]
-    const int32_t* pair_ce;   // [P]       (chunk << 8) | expert
-    const uint32_t* tmask;    // [C, E]
-    __nv_bfloat16* hbuf;      // [C*E*N, d_e] gated activations of every pair
-    float* partA;             // [grid][2][N*128] split-K partial sums (expert-in GEMM)
-    float* partB;             // [grid][2][N*128] split-expert partial sums (expert-out GEMM)
-    // counters, two sets chosen by launch parity (each launch zeroes the other set)
+    const uint32_t* tmask;    // [C, E] chunk token masks
+    const int32_t* gcounts;   // [NGr] size of each group's expert set
+    const int32_t* goffsets;  // [NGr + 1]
+    const int32_t* gpair;     // [P] (group << 8) | expert, by group, experts ascending
+    __nv_bfloat16* hbuf;      // [P][N][d_e] gated activations h'
+    float* partA;             // [grid][2][N*128] split-K partial sums (expert-in)
+    float* partB;             // [grid][2][N*128] split-expert partial sums (expert-out)
     uint32_t* cntA;           // [2][cnt_a_len] blocks that published an expert-in partial
     uint32_t* readyA;         // [2][cnt_a_len] blocks whose rows of h' are written
     uint32_t* cntB;           // [2][cnt_b_len] blocks that published an expert-out partial
-    long long cnt_a_len;      // C*E*MT: expert-in units
-    long long cnt_b_len;      // C*RT: expert-out units
+    long long cnt_a_len;      // NGr*E*MT
+    long long cnt_b_len;      // NGr*RT
     Ctl* ctl;
     __nv_bfloat16* y;         // [T, d_h]
-    int T, d_h, E, d_e, n, N, C;
-    int KB;    // d_h / 64: k-blocks of one expert-in unit
-    int MT;    // d_e / 128: 128-row tiles of one expert's W_in
-    int RT;    // d_h / 128: 128-row tiles of y
-    int KBe;   // d_e / 64: k-blocks of one expert in the expert-out GEMM
-    int fuse_union;   // 1 when C == 1: each block forms the union itself from gates
-    int skip_flag_unit;   // test support: unit whose h' is never announced ready (-1: off)
-    unsigned long long* trace;   // optional [grid][16] globaltimer stamps (nullptr: off)
+    int T, d_h, E, d_e, n;
+    int N;     // tokens per MMA: 128 or 256
+    int NT;    // tokens per group: (N / n) * n
+    int NGr;   // groups
+    int KB, MT, RT, KBe;
+    int skip_flag_unit;       // test support: unit whose h' is never announced ready (-1: off)
     unsigned long long wait_ns;
-    unsigned long long shape_key;   // the workspace layout this launch expects (Ctl::shape_key)
+    unsigned long long shape_key;
+    unsigned long long* trace;   // optional [grid][64] globaltimer stamps (nullptr: off)
 };
-
-// maps: x, W_in, W_out (2-D, bf16, 128-byte swizzle, boxes {64,N}, {64,128}, {64,128})
-cudaError_t launch_forward_tc(const TcArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s);
-size_t forward_tc_smem_bytes();
+// maps: x [T, d_h] (box {64, N}), W_in [E*d_e, d_h] and W_out [E*d_h, d_e] (box
+// {64, 128}), h' [P*N, d_e] (box {64, N}); 2-D, bf16, 128-byte swizzle
+cudaError_t launch_forward_group(const GrArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s);
 
 // Arguments of the single-chunk forward (see forward_decode.cu): expert-in
 // units are (union expert, 128-row tile of W_in) split along K over a pair of
@@ -77,6 +82,11 @@ size_t forward_tc_smem_bytes();
 // reduced in two passes.
 struct DcArgs {
     const float* gates;       // [T, E], T <= n
+    // the caller's union tables of the chunk (counts [1], idx [E], tmask [E]), or
+    // all nullptr: the kernel forms the union from the gates
+    const int32_t* counts_in;
+    const int32_t* idx_in;
+    const uint32_t* tmask_in;
     __nv_bfloat16* y;         // [T, d_h]
     __nv_bfloat16* hbuf;      // [E slots][N][d_e] gated activations h'
     uint32_t* readyA;         // [2][E] halves of an expert slot written, by launch parity

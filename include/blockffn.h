@@ -153,6 +153,13 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  * Gating source, exactly one of:
  *   gates != NULL : injected gates [T, E] fp32 (W_r, b_r, gamma ignored, must be NULL);
  *   gates == NULL : the router runs first (W_r, gamma required, b_r optional, eps).
+ * Union tables (counts [C] int32, idx [C, E] int32, tmask [C, E] uint32, C =
+ * ceil(T / n)), either all NULL -- the union is formed from the gates -- or all
+ * given, exactly as blockffn_chunk_union returns them for these gates and n
+ * (injected gates only).  Given tables replace the union step: the token masks
+ * decide which experts run and which tokens are kept; counts and idx are checked
+ * against the masks on the device, and a mismatch records
+ * BLOCKFFN_ERR_INVALID_ARG in the status word (detail 11) and computes nothing.
  * W_in [E, d_e, d_h] and W_out [E, d_h, d_e] in dtype dt; y [T, d_h] in dtype dt is
  * fully overwritten (rows of tokens with no active expert are exact zeros).
  * workspace: ws_bytes >= blockffn_forward_workspace_bytes(...), reset once with
@@ -167,14 +174,20 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  *   fp32: any d_h, d_e >= 1.
  * Arithmetic: bf16 inputs, fp32 accumulation; the gated Swish activations are
  * rounded to bf16 between the two GEMMs; y is rounded once to dt.
+ * Kernels: one chunk (T <= n, bf16, d_h % 256 == 0) runs the single-chunk
+ * cluster kernel; several chunks run the group kernel, which takes whole chunks
+ * 256 tokens at a time (128 when T <= 128) and runs each expert of the group's
+ * union once over all of them, masking every token by its own chunk's mask.
  * Ordering: stream-ordered like any kernel launch.  The single-chunk bf16 kernel
- * (T <= n) is launched as a programmatic dependent of the preceding kernel on
- * the stream: its blocks may start while that kernel finishes, but they set up
+ * is launched as a programmatic dependent of the preceding kernel on the
+ * stream: its blocks may start while that kernel finishes, but they set up
  * only their own on-chip state before waiting for it to complete, so inputs
- * produced by the preceding kernel (x, gates, weights) are read only after it.
+ * produced by the preceding kernel (x, gates, tables, weights) are read only
+ * after it.
  */
 blockffn_status blockffn_forward(const void* x, const float* gates, const void* W_r,
                                  const float* b_r, const float* gamma, float eps,
+                                 const int32_t* counts, const int32_t* idx, const uint32_t* tmask,
                                  const void* W_in, const void* W_out, int T, int d_h,
                                  int E, int d_e, int n, blockffn_dtype dt, void* y,
                                  void* workspace, size_t ws_bytes, void* stream);
@@ -211,8 +224,9 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
  * blockffn_get_device_status -- synchronize stream, then read the device status
  * word of a workspace: BLOCKFFN_OK, or the first device-side error recorded
  * (BLOCKFFN_ERR_TIMEOUT, BLOCKFFN_ERR_WORKSPACE).  detail (may be NULL) receives
- * a code naming the wait that ran out (1-9), or 10 for a workspace bound to
- * other shapes or another gating mode.  Returns BLOCKFFN_ERR_CUDA if the
+ * a code naming the wait that ran out (1-9), 10 for a workspace bound to
+ * other shapes or another gating mode, or 11 for union tables whose counts or
+ * index lists disagree with their token masks.  Returns BLOCKFFN_ERR_CUDA if the
  * synchronization itself failed.
  */
 blockffn_status blockffn_get_device_status(const void* workspace, void* stream,

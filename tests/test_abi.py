@@ -73,8 +73,8 @@ def test_status_strings(lib):
 def test_forward_rejects_bad_shapes_on_host(lib, T, d_h, E, d_e, n, dt):
     L = lib.lib
     assert L.blockffn_forward_workspace_bytes(T, d_h, E, d_e, n, dt, 0) == 0
-    st = L.blockffn_forward(16, 16, None, None, None, 0.0, 16, 16, T, d_h, E, d_e, n, dt, 16, 16,
-                            1 << 30, None)
+    st = L.blockffn_forward(16, 16, None, None, None, 0.0, None, None, None, 16, 16, T, d_h, E, d_e,
+                            n, dt, 16, 16, 1 << 30, None)
     assert st in (lib.ERR_INVALID_ARG, lib.ERR_UNSUPPORTED)
     assert L.blockffn_last_error_message()
 
@@ -83,13 +83,28 @@ def test_forward_gating_source_is_exclusive(lib):
     L = lib.lib
     # (T = 32 > 0: with T = 0 the call is a no-op before this check)
     # gates and router weights together
-    st = L.blockffn_forward(16, 16, 16, None, None, 0.0, 16, 16, 32, 2048, 64, 128, 32, 1, 16, 16,
-                            1 << 30, None)
+    st = L.blockffn_forward(16, 16, 16, None, None, 0.0, None, None, None, 16, 16, 32, 2048, 64, 128,
+                            32, 1, 16, 16, 1 << 30, None)
     assert st == lib.ERR_INVALID_ARG
     # neither
-    st = L.blockffn_forward(16, None, None, None, None, 0.0, 16, 16, 32, 2048, 64, 128, 32, 1, 16,
-                            16, 1 << 30, None)
+    st = L.blockffn_forward(16, None, None, None, None, 0.0, None, None, None, 16, 16, 32, 2048, 64,
+                            128, 32, 1, 16, 16, 1 << 30, None)
     assert st == lib.ERR_INVALID_ARG
+
+
+def test_forward_union_tables_all_or_none(lib):
+    """counts, idx and tmask come together or not at all, only with injected gates,
+    and 16-byte aligned; each refusal is made on the host."""
+    L = lib.lib
+    args = (16, 16, 32, 2048, 64, 128, 32, 1, 16, 16, 1 << 30, None)
+    # two of the three
+    assert L.blockffn_forward(16, 16, None, None, None, 0.0, 16, 16, None, *args) == lib.ERR_INVALID_ARG
+    assert L.blockffn_forward(16, 16, None, None, None, 0.0, None, None, 16, *args) == lib.ERR_INVALID_ARG
+    # with the router
+    assert L.blockffn_forward(16, None, 16, None, 16, 0.0, 16, 16, 16, *args) == lib.ERR_INVALID_ARG
+    assert b"injected" in L.blockffn_last_error_message()
+    # misaligned table
+    assert L.blockffn_forward(16, 16, None, None, None, 0.0, 16, 20, 16, *args) == lib.ERR_INVALID_ARG
 
 
 def test_union_and_route_reject_bad_args(lib):
@@ -122,5 +137,5 @@ def test_empty_inputs_are_no_ops(lib):
     # T = 0: nothing to do, nothing launched, no pointer needed
     assert L.blockffn_chunk_union(None, 0, 64, 32, None, None, None, None) == lib.OK
     assert L.blockffn_route(None, None, None, None, 0.0, 0, 64, 16, 1, None, None) == lib.OK
-    assert L.blockffn_forward(None, 16, None, None, None, 0.0, None, None, 0, 2048, 64, 128, 32,
-                              1, None, None, 0, None) == lib.OK
+    assert L.blockffn_forward(None, 16, None, None, None, 0.0, None, None, None, None, None, 0, 2048,
+                              64, 128, 32, 1, None, None, 0, None) == lib.OK

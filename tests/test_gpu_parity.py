@@ -184,6 +184,44 @@ def test_forward_single_chunk_wide_experts(bffn, T, n, d_h, E, d_e):
     assert_close(y, oracle_y(w, g), "bf16", f"single chunk T{T} n{n} d_h{d_h} E{E} d_e{d_e}")
 
 
+@pytest.mark.parametrize("T,n,d_h,E,d_e,dt", [
+    (32, 32, 2048, 64, 128, "bf16"),    # one chunk: the single-chunk kernel reads the tables
+    (300, 32, 512, 64, 128, "bf16"),    # several groups: the group plan reads the token masks
+    (70, 8, 256, 16, 256, "bf16"),      # short chunks, N = 128 groups, wide experts
+    (40, 16, 256, 16, 64, "f32"),       # the fp32 path
+])
+def test_forward_with_caller_union_tables(bffn, T, n, d_h, E, d_e, dt):
+    """blockffn_chunk_union's tables fed to blockffn_forward: the same bits as the
+    forward that forms the union itself, and the oracle's result."""
+    w = wl.make_injected("tables", T, n, d_h, E, d_e, dt, "markov80", seed=T + n)
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    x, W_in, W_out = dev(w.x, tdt), dev(w.W_in, tdt), dev(w.W_out, tdt)
+    g = dev(w.gates, torch.float32)
+    tables = bffn.chunk_union(g, n)
+    y_tab = bffn.forward(x, W_in, W_out, n, gates=g, union=tables)
+    y_own = bffn.forward(x, W_in, W_out, n, gates=g)
+    torch.cuda.synchronize()
+    assert torch.equal(y_tab, y_own), "tables given vs formed: results differ"
+    assert_close(to_np64(y_tab), oracle_y(w, w.gates.astype(np.float64)), dt, f"tables T{T} n{n}")
+
+
+@pytest.mark.parametrize("T", [32, 300])
+def test_forward_refuses_inconsistent_union_tables(bffn, T):
+    """An index list that disagrees with its token masks is refused on the device
+    (status BLOCKFFN_ERR_INVALID_ARG, detail 11) and nothing is written."""
+    w = wl.make_injected("badtab", T, 32, 512 if T > 32 else 2048, 64, 128, "bf16", "markov80", seed=5)
+    x, W_in, W_out = dev(w.x, torch.bfloat16), dev(w.W_in, torch.bfloat16), dev(w.W_out, torch.bfloat16)
+    g = dev(w.gates, torch.float32)
+    counts, idx, tmask = bffn.chunk_union(g, 32)
+    idx = idx.clone()
+    idx[0, 0] = (idx[0, 0] + 1) % w.E           # names the wrong expert
+    ws = bffn.Workspace.for_shapes(T, w.d_h, w.E, w.d_e, 32, torch.bfloat16, False)
+    y = torch.full((T, w.d_h), 5.0, dtype=torch.bfloat16, device="cuda")
+    bffn.forward(x, W_in, W_out, 32, gates=g, y=y, workspace=ws, union=(counts, idx, tmask))
+    assert bffn.device_status(ws) == (1, 11)
+    assert torch.all(y == 5.0)
+
+
 def test_workspace_bound_to_its_shapes(bffn):
     """A workspace is bound to the shapes and gating mode of its first call after a
     reset: a call with other shapes is refused on the device (status
