@@ -258,7 +258,7 @@ def union_stats(gates: np.ndarray, n: int):
     return sizes, distinct
 
 
-def measure_workloads(dev, stream, with_oracle: bool) -> dict:
+def measure_workloads(dev, stream, with_oracle: bool, which=("batch16", "seq4096", "sweep")) -> dict:
     """The other configurations, each timed on the device as CUDA-graph replays of
     the call a user makes, beside the same-size dense FFN (torch bf16 matmuls):
 
@@ -269,7 +269,6 @@ def measure_workloads(dev, stream, with_oracle: bool) -> dict:
     Inputs larger than L2 between replays: rotating copies (batch16, seq4096) or
     weights of 256 MiB (sweep)."""
     import torch
-    import chunk_sparse_moe_b200 as bffn
     dt = torch.bfloat16
     d = lambda a, t=dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev, t)
     out = {}
@@ -280,7 +279,21 @@ def measure_workloads(dev, stream, with_oracle: bool) -> dict:
         Wo = W_out.permute(1, 0, 2).reshape(d_h, E * d_e).contiguous()
         return graph_us([lambda x=x: torch.nn.functional.silu(x @ Wi.t()) @ Wo.t() for x in x_list], stream)
 
-    # ---- batch16
+    if "batch16" in which:
+        out["batch16"] = _batch16(dev, stream, d, dense_us, with_oracle)
+    if "seq4096" in which:
+        out["seq4096"] = _seq4096(dev, stream, d, dense_us, with_oracle)
+    if "sweep" in which:
+        out["sweep"] = _sweep(dev, stream, d, dense_us)
+    return out
+
+
+def _batch16(dev, stream, d, dense_us, with_oracle):
+    """16 independent 32-token chunks in one call (the group kernel); 4 rotating
+    copies of the weights and x (256 MiB of weights > L2)."""
+    import torch
+    import chunk_sparse_moe_b200 as bffn
+    dt = torch.bfloat16
     w = wl.batch16()
     R = 4
     W_in = [d(w.W_in) for _ in range(R)]
@@ -293,22 +306,31 @@ def measure_workloads(dev, stream, with_oracle: bool) -> dict:
                    for k in range(R)], stream)
     assert bffn.device_status(ws) == (0, 0)
     sizes, distinct = union_stats(w.gates, w.n)
+    gsizes, _ = union_stats(w.gates, 256)
     flops = sum(sizes) * w.n * 4 * w.d_h * w.d_e
     nbytes = distinct * 2 * w.d_h * w.d_e * 2 + 2 * w.T * w.d_h * 2 + w.T * w.E * 4
-    out["batch16"] = {
+    out = {
         "what": "16 chunks x 32 tokens, d_h 2048, E 64, d_e 128, bf16, Markov80 gates per sequence",
         "us_per_call": us, "tokens_per_s": w.T / (us * 1e-6),
         "union_experts_sum": sum(sizes), "distinct_experts": distinct,
         "algorithmic_bytes": nbytes, "union_flops": flops,
+        "executed_flops": sum(gsizes) * 256 * 4 * w.d_h * w.d_e,
         "roofline": roofline_of(nbytes, flops, us),
         "dense_ffn_us": dense_us(xs, W_in[0], W_out[0]),
     }
     if with_oracle:
-        out["batch16"]["cpu_baseline"] = oracle_sample(w, 32, False)
+        out["cpu_baseline"] = oracle_sample(w, 32, False)
     del W_in, W_out, xs, ws
     torch.cuda.empty_cache()
+    return out
 
-    # ---- seq4096 (router in the call)
+
+def _seq4096(dev, stream, d, dense_us, with_oracle):
+    """4096 tokens, router + union + forward in one call; 2 rotating copies of
+    the weights, router and x (160 MiB > L2)."""
+    import torch
+    import chunk_sparse_moe_b200 as bffn
+    dt = torch.bfloat16
     w = wl.seq4096()
     R = 2
     W_in = [d(w.W_in) for _ in range(R)]
@@ -323,23 +345,33 @@ def measure_workloads(dev, stream, with_oracle: bool) -> dict:
     assert bffn.device_status(ws) == (0, 0)
     gates = bffn.route(xs[0], W_r[0], gam, w.eps, b_r=b_r).cpu().numpy()
     sizes, distinct = union_stats(gates, w.n)
+    gsizes, _ = union_stats(gates, 256)
     flops = sum(sizes) * w.n * 4 * w.d_h * w.d_e + 2 * w.T * w.d_h * w.E
     nbytes = (distinct * 2 * w.d_h * w.d_e * 2 + 2 * w.T * w.d_h * 2 + w.E * w.d_h * 2 + w.T * w.E * 4)
-    out["seq4096"] = {
+    out = {
         "what": "4096 tokens (128 chunks of 32), router with bias -0.8 sigma, AR(1) x, d_h 2048, E 64, "
                 "d_e 128, bf16; route + union + forward in the call",
         "us_per_call": us, "tokens_per_s": w.T / (us * 1e-6),
         "mean_union_experts": float(np.mean(sizes)), "distinct_experts": distinct,
+        "mean_group_union_experts": float(np.mean(gsizes)),
         "algorithmic_bytes": nbytes, "union_flops": flops,
+        "executed_flops": sum(gsizes) * 256 * 4 * w.d_h * w.d_e,
         "roofline": roofline_of(nbytes, flops, us),
         "dense_ffn_us": dense_us(xs, W_in[0], W_out[0]),
     }
     if with_oracle:
-        out["seq4096"]["cpu_baseline"] = oracle_sample(w, 16, True)
+        out["cpu_baseline"] = oracle_sample(w, 16, True)
     del W_in, W_out, W_r, xs, ws
     torch.cuda.empty_cache()
+    return out
 
-    # ---- sweep: d_h 4096, E 128, the whole sequence as one-chunk decode calls
+
+def _sweep(dev, stream, d, dense_us):
+    """d_h 4096, E 128: every chunk of the 4096-token sequence as its own decode
+    call, n in {1, 8, 32}, four gate regimes (256 MiB of weights > L2)."""
+    import torch
+    import chunk_sparse_moe_b200 as bffn
+    dt = torch.bfloat16
     base = wl.sweep(32, "all_on", T=32)
     W_in, W_out = d(base.W_in), d(base.W_out)
     rows = []
@@ -368,11 +400,10 @@ def measure_workloads(dev, stream, with_oracle: bool) -> dict:
                          "dense_ffn_us": dense_cache[n],
                          "speedup_vs_dense": dense_cache[n] / us})
         del ws
-    out["sweep"] = {"what": "d_h 4096, E 128, d_e 128, bf16, T 4096: every chunk of the sequence as its own "
-                            "decode call (graph of consecutive calls), mean per call; dense = the same-size "
-                            "dense FFN on n tokens (torch bf16)",
-                    "rows": rows}
-    return out
+    return {"what": "d_h 4096, E 128, d_e 128, bf16, T 4096: every chunk of the sequence as its own decode "
+                    "call (a graph of the consecutive calls), mean per call; dense = the same-size dense FFN "
+                    "on n tokens (torch bf16)",
+            "rows": rows}
 
 
 def run_reference(args, world, rank):
@@ -403,6 +434,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the batch16 / seq4096 / sweep measurements")
+    ap.add_argument("--workloads", default="batch16,seq4096,sweep",
+                    help="comma list of the other workloads to measure (batch16, seq4096, sweep)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -664,7 +697,8 @@ def main():
         cb = cpu_baseline()
     other = None
     if not args.no_workloads:
-        other = measure_workloads(dev, stream, with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
+        other = measure_workloads(dev, stream, with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline,
+                                  which=set(args.workloads.split(",")))
 
     if rank == 0:
         value = world * T * args.steps / (elapsed_ms * 1e-3)

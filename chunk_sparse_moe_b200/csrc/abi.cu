@@ -125,7 +125,7 @@ enum class Path { F32, Decode, Group };
 struct Layout {
     Path path;
     size_t ctl, counts, offsets, idx, tmask, pair_ce, gcounts, goffsets, gpair, gates;
-    size_t cntA, readyA, cntB, partA, partB, hbuf;
+    size_t readyA, cntB, partB, hbuf;
     size_t total;
     int C;               // chunks
     int N;               // tokens per MMA
@@ -169,7 +169,7 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         return o;
     };
     L.ctl = L.counts = L.offsets = L.idx = L.tmask = L.pair_ce = L.gcounts = L.goffsets = L.gpair = 0;
-    L.gates = L.cntA = L.readyA = L.cntB = L.partA = L.partB = L.hbuf = 0;
+    L.gates = L.readyA = L.cntB = L.partB = L.hbuf = 0;
     L.NG = L.NT = L.NGr = 0;
     const size_t C = (size_t)L.C;
     L.ctl = take(sizeof(Ctl));
@@ -203,10 +203,8 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         L.gcounts = take(NGr * 4);
         L.goffsets = take((NGr + 1) * 4);
         L.gpair = take(Pm * 4);
-        L.cntA = take(2 * Pm * L.MT * 4);
         L.readyA = take(2 * Pm * L.MT * 4);
         L.cntB = take(2 * NGr * L.RT * 4);
-        L.partA = take((size_t)G * 2 * L.N * 128 * 4);
         L.partB = take((size_t)G * 2 * L.N * 128 * 4);
         L.hbuf = take(Pm * L.N * d_e * 2);
     }
@@ -421,7 +419,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.skip_unit = g_skip_flag.load();
         da.wait_ns = g_wait_ns.load();
         da.trace = g_trace.load();
-        da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1});
+        da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1, Gd});
         // A cluster launch cannot also be cooperative; the grid is sized to the
         // clusters that can be resident at once, and every wait is bounded.
         e = launch_forward_decode(da, dmaps, Gd, s);
@@ -449,9 +447,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.goffsets = goffsets;
     a.gpair = gpair;
     a.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
-    a.partA = reinterpret_cast<float*>(ws + L.partA);
     a.partB = reinterpret_cast<float*>(ws + L.partB);
-    a.cntA = reinterpret_cast<uint32_t*>(ws + L.cntA);
     a.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
     a.cntB = reinterpret_cast<uint32_t*>(ws + L.cntB);
     a.cnt_a_len = L.Pmax * L.MT;
@@ -472,7 +468,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.KBe = L.KBe;
     a.skip_flag_unit = g_skip_flag.load();
     a.wait_ns = g_wait_ns.load();
-    a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2});
+    a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2, G});
     a.trace = g_trace.load();
     e = launch_forward_group(a, maps, G, s);
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "group forward launch");
@@ -573,7 +569,7 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     da.skip_unit = -1;
     da.wait_ns = g_wait_ns.load();
     da.trace = nullptr;
-    da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)BLOCKFFN_BF16, 0, 3});
+    da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)BLOCKFFN_BF16, 0, 3, Gd});
     e = launch_forward_decode(da, dmaps, Gd, s);
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "no-allocation forward launch");
 }

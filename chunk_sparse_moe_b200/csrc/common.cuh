@@ -39,15 +39,19 @@ enum : int32_t {
 struct Ctl {
     int32_t status;        // first device-side error (sticky until reset)
     int32_t detail;        // which wait / check
-    uint32_t epoch;        // number of completed forward launches (flag stamp)
-    uint32_t done;         // thread blocks of the current launch that finished
+    uint32_t unused_[2];
     uint32_t issued[2];    // by launch parity: blocks that issued their last expert-in load
     // The shapes, dtype, gating mode and kernel the workspace's layout was made
     // for, claimed by the first launch after a reset (0 = not yet bound).  A
     // launch whose key differs records kErrWorkspace and computes nothing: its
     // counters and tables would sit at other offsets.
     unsigned long long shape_key;
-    uint32_t pad[56];
+    // One ticket per thread block of every launch on this workspace: block b of
+    // launch k draws a ticket in [k*G, (k+1)*G) (G = the launch's grid, fixed for
+    // a workspace by its shape key), so ticket / G is the launch's index with one
+    // atomic and no end-of-launch bookkeeping.  64 bits: it never wraps.
+    unsigned long long ticket;
+    uint32_t pad[54];
 };
 static_assert(sizeof(Ctl) == 256, "control block is 256 bytes");
 

@@ -273,21 +273,15 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     griddep_wait();
     if (threadIdx.x == 0) {
         griddep_launch_dependents();
+        // Three independent control-block accesses, issued back to back so their
+        // round trips overlap: the sticky status, this block's launch ticket (the
+        // launch index is ticket / grid) and the workspace's shape key.
         const int32_t st0 = __ldcg(&a.ctl->status);
-        // acquire: the read is done before this block's count below is seen
-        const uint32_t ep0 = ld_acquire_gpu(&a.ctl->epoch);
+        const unsigned long long tk = atomicAdd(&a.ctl->ticket, 1ull);
+        const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
+        const uint32_t ep0 = (uint32_t)(tk / gridDim.x);
         if (blockIdx.x == 0) a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;   // the next launch's counter
         sh.epoch = ep0;
-        // The last block to read the launch counter advances it for the next
-        // launch (every block of this one has read it by then; the next launch
-        // sees the new value because it reads it only after this one has
-        // completed: stream order, or its griddep_wait).
-        const uint32_t done0 = atomicAdd(&a.ctl->done, 1u);
-        const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
-        if (done0 == (uint32_t)(gridDim.x - 1)) {
-            a.ctl->done = 0u;
-            a.ctl->epoch = ep0 + 1u;
-        }
         const bool key_ok = key0 == 0ull || key0 == a.shape_key;
         if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
         sh.abort = st0 != 0 || !key_ok;
@@ -387,7 +381,6 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // ------------------------------------------------------ TMA producer --
         if (lane == 0 && !sh.abort) {
             const uint64_t pol_stream = policy_evict_first();
-            const uint64_t pol_keep = policy_evict_last();
             long long i = 0;
             RingPos rp;
             bool stop = false;
@@ -401,9 +394,8 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         break;
                     }
                     uint8_t* w = smem + rp.st * kRsStageBytes;
-                    mbar_arrive_expect_tx(&sh.full_w[rp.st], kRsWBytes + N * 256);
+                    mbar_arrive_expect_tx(&sh.full_w[rp.st], kRsWBytes);
                     tma_load_3d(w, &tm_win, &sh.full_w[rp.st], 0, e * a.d_e + mt * 128, kb, pol_stream);
-                    tma_load_3d(w + kRsWBytes, &tm_x, &sh.full_w[rp.st], 0, 0, kb, pol_keep);
                     if (i == 0) RS_TRACE(kRtFirstLoad);
                 }
             }
@@ -540,22 +532,29 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         if (leader) umma_commit(&sh.mma_done);
         __syncwarp();
     } else if (warp == 2) {
-        // ------------------------------------------------------- h' loader --
-        // A stages carry no h': lane 0 just arrives.  Before the first expert-out
-        // tile the warp waits (bounded) until every expert slot's h' is counted in;
-        // then lane 0 moves each tile's [N x 64] h' slice with one TMA load, which
-        // lands in the same 128-byte-swizzled layout as the weight tile's operand.
-        const long long nAt = (long long)wk.nA * KP;
+        // ------------------------------------------------- activation loader --
+        // An expert-in stage's activations are the chunk's two x k-blocks of the
+        // stage (lane 0 issues them, so the weight tiles and the activation tiles
+        // come from two issuing threads: one thread issues bulk copies at a bounded
+        // rate).  Before the first expert-out tile the warp waits (bounded) until
+        // every expert slot's h' is counted in; then lane 0 moves each tile's
+        // [N x 64] h' slice with one TMA load, which lands in the same
+        // 128-byte-swizzled layout as the weight tile's operand.
         long long i = 0;
         RingPos rp;
         int stop = sh.abort != 0;
         if (lane == 0) {
-            for (; i < nAt; ++i, rp.advance()) {
-                if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
-                    stop = 1;
-                    break;
+            const uint64_t pol_keep = policy_evict_last();
+            for (int ua = 0; ua < wk.nA && !stop; ++ua) {
+                for (int t = 0; t < KP; ++t, ++i, rp.advance()) {
+                    if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
+                        stop = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 256));
+                    tma_load_3d(smem + rp.st * kRsStageBytes + kRsWBytes, &tm_x, &sh.full_h[rp.st], 0, 0,
+                                2 * (wk.hk * KP + t), pol_keep);
                 }
-                mbar_arrive(&sh.full_h[rp.st]);
             }
         }
         stop = __shfl_sync(0xffffffffu, stop, 0);
@@ -600,10 +599,14 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     tma_load_3d(smem + rp.st * kRsStageBytes + kRsWBytes, &tm_h, &sh.full_h[rp.st], 0, bc.s * N,
                                 2 * bc.kb, pol);
                 }
-                // no copy into this block's shared memory outlives it
-                for (long long q = i - kRsStages < nAt ? nAt : i - kRsStages; q < i; ++q)
-                    wait_bar_drain(&sh.full_h[q % kRsStages], (uint32_t)((q / kRsStages) & 1), limit, a.ctl);
             }
+        }
+        if (lane == 0) {
+            // no copy into this block's shared memory outlives it: the last ring's
+            // worth of stages this warp filled (x or h'; an earlier stage's slot was
+            // only refilled after the MMAs had read it, so its copy had landed)
+            for (long long q = i - kRsStages < 0 ? 0 : i - kRsStages; q < i; ++q)
+                wait_bar_drain(&sh.full_h[q % kRsStages], (uint32_t)((q / kRsStages) & 1), limit, a.ctl);
         }
     } else {
         // --------------------------------------------------------- epilogue --

@@ -23,20 +23,21 @@
 // bit_j is token t_j's bit in its chunk's token mask (the chunk union tables).
 //
 // Schedule.  One persistent block per SM (cooperative launch: all resident).  The
-// A work (pairs x 128-row tiles x 64-wide k-blocks) and the B work (groups x
-// 128-row tiles of y x (expert, k-block)) are each cut into equal contiguous
-// ranges of 16 KB weight tiles, one range of each per block, so every SM streams
-// the same number of weight bytes and A tiles come before B tiles everywhere.  A
-// unit split across blocks is finished by each contributor for its share of the
-// rows, summing the partials in block order (a fixed order: results do not depend
-// on timing).  An expert-out tile waits, with a bounded spin, until every
-// contributor of the expert-in unit it reads has written its rows of h'.
+// A work is dealt out in whole units (a pair's 128-row tile of W_in_e over all of
+// d_h), an equal count per block, so h' comes straight from one accumulator.  The
+// B work (groups x 128-row tiles of y x (expert, k-block)) is cut into equal
+// contiguous ranges of 16 KB weight tiles, one per block; an expert-out unit split
+// across blocks is finished by each contributor for its share of the rows,
+// summing the partials in block order (a fixed order: results do not depend on
+// timing).  A tiles come before B tiles everywhere, and an expert-out tile waits,
+// with a bounded spin, until the block owning the expert-in unit it reads has
+// written that unit's h'.
 //
-// Roles (224 threads): warp 0 issues the weight/activation TMA loads, warp 1
-// issues the MMAs (the whole warp runs the loop, one elected lane issues), warp 2
-// owns TMEM and loads h' tiles by TMA once their flag is set, warps 3-6 drain the
-// accumulators (TMEM -> registers, 32 columns at a time) and do the split
-// reductions, Swish, gate, mask and stores.
+// Roles (224 threads): warp 0 issues the weight-tile TMA loads, warp 1 issues
+// the MMAs (the whole warp runs the loop, one elected lane issues), warp 2 owns
+// TMEM and issues the activation-tile TMA loads (x, or h' once its flag is set),
+// warps 3-6 drain the accumulators (TMEM -> registers, 32 columns at a time) and
+// do the split reductions, Swish, gate, mask and stores.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -54,6 +55,8 @@ constexpr int kGrWBytes = 128 * 128;            // weight tile: 128 rows x 64 bf
 constexpr int kGrMaxE = 256;
 constexpr int kGrMaxContrib = 160;              // >= blocks per launch (one per SM)
 constexpr int kGrSmemBudget = 200 * 1024;       // pipeline stages
+// epilogue output staging: two [32 tokens][128 rows] bf16 slices (8 KB each)
+constexpr int kGrOutStageBytes = 2 * 32 * 128 * 2;
 
 template <int N>
 struct GrCfg {
@@ -71,6 +74,7 @@ struct GrShared {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
+    uint64_t a_pub;                        // this block's expert-in results are announced
     uint32_t tmem_base;
     volatile int abort;
     int abort0;                            // abort as set before the first block barrier
@@ -190,7 +194,8 @@ __device__ __forceinline__ float gr_swish(float z) { return __fdividef(z, 1.0f +
 enum : int {
     kGtStart = 0, kGtPrologue = 1, kGtFirstLoad = 2, kGtLastALoad = 3, kGtLastACommit = 4,
     kGtAFlushed = 5, kGtFirstFlag = 6, kGtLastBCommit = 7, kGtEpiEnd = 8, kGtEnd = 9,
-    kGtFirstAcc = 10, kGtFirstBLoad = 11, kGtLastLoad = 12, kGtSlots = 64
+    kGtFirstAcc = 10, kGtFirstBLoad = 11, kGtLastLoad = 12, kGtADrained = 13, kGtAnnounce = 14,
+    kGtFirstSlice = 15, kGtSlots = 64
 };
 #define GR_TRACE(slot) \
     do { if (a.trace) a.trace[(size_t)blockIdx.x * kGtSlots + (slot)] = globaltimer_ns(); } while (0)
@@ -209,6 +214,8 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     GrShared<N>& sh = *reinterpret_cast<GrShared<N>*>(smem + kStages * kStageBytes);
+    __nv_bfloat16* ostage = reinterpret_cast<__nv_bfloat16*>(
+        (reinterpret_cast<uintptr_t>(&sh + 1) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, cta = blockIdx.x;
 
@@ -224,11 +231,13 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             mbar_init(&sh.acc_empty[s], 4);
         }
         mbar_init(&sh.mma_done, 1);
+        mbar_init(&sh.a_pub, 1);
         fence_mbar_init();
         // written by earlier launches only: plain L2 loads
         const int32_t st0 = __ldcg(&a.ctl->status);
-        const uint32_t ep0 = __ldcg(&a.ctl->epoch);
+        const unsigned long long tk = atomicAdd(&a.ctl->ticket, 1ull);   // launch index = ticket / grid
         const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
+        const uint32_t ep0 = (uint32_t)(tk / gridDim.x);
         const bool key_ok = key0 == 0ull || key0 == a.shape_key;
         if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
         sh.abort = st0 != 0 || !key_ok;
@@ -250,14 +259,17 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 
     const uint32_t tmem = sh.tmem_base;
     const int P = a.goffsets[a.NGr];
-    const uint32_t stamp = sh.epoch + 1u;
     const int par = (int)(sh.epoch & 1u);
-    uint32_t* const cntA = a.cntA + (size_t)par * a.cnt_a_len;
     uint32_t* const readyA = a.readyA + (size_t)par * a.cnt_a_len;
     uint32_t* const cntB = a.cntB + (size_t)par * a.cnt_b_len;
-    const long long NA = (long long)P * a.MT * a.KB;
     const long long NB = (long long)P * a.RT * a.KBe;
-    const long long aLo = NA > 0 ? gr_range_lo(NA, G, cta) : 0, aHi = NA > 0 ? gr_range_lo(NA, G, cta + 1) : 0;
+    // Expert-in work goes to blocks in whole units (a unit is one pair's 128-row
+    // tile of W_in_e over all of d_h: KB tiles), so no expert-in result is ever
+    // split and h' is written straight from the accumulator; block i takes units
+    // [i*UA/G, (i+1)*UA/G).  Expert-out work is cut into equal tile ranges.
+    const long long UA = (long long)P * a.MT;
+    const long long aLo = UA > 0 ? gr_range_lo(UA, G, cta) * a.KB : 0;
+    const long long aHi = UA > 0 ? gr_range_lo(UA, G, cta + 1) * a.KB : 0;
     const long long bLo = NB > 0 ? gr_range_lo(NB, G, cta) : 0, bHi = NB > 0 ? gr_range_lo(NB, G, cta + 1) : 0;
     // waits on other blocks run out after wait_ns; waits on this block's own
     // pipeline are downstream of those and get twice as long, so the first
@@ -267,11 +279,11 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer --
-        // A group's x tile is read once per expert of its set: kept in L2.  Weight
-        // tiles are read once per group that uses the expert, by blocks that run at
-        // about the same time: the normal policy.
+        // Weight tiles only (the activation tiles come from warp 2: one thread
+        // issues bulk copies at a bounded rate, so two issuers keep the stages
+        // full).  A weight tile is read once per group that uses the expert, by
+        // blocks that run at about the same time: the normal L2 policy.
         const uint64_t pol_weights = policy_evict_normal();
-        const uint64_t pol_keep = policy_evict_last();
         GrIter it;
         it.init(aLo, aHi, bLo, bHi);
         GrSeg sg;
@@ -290,8 +302,13 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     const long long local = sg.lo - sg.first;
                     sidx = (int)(local / a.KBe);
                     kb = (int)(local - (long long)sidx * a.KBe);
+                    // no expert-out copy is in flight while the block announces its
+                    // h' (a fence waits for the block's bulk copies in flight)
+                    if (sg.lo == bLo && aHi > aLo &&
+                        !wait_bar(&sh.a_pub, 0u, limit, &sh.abort, a.ctl, kWaitEmpty))
+                        stop = true;
                 }
-                for (long long j = sg.lo; j < sg.hi; ++j, ++i) {
+                for (long long j = sg.lo; j < sg.hi && !stop; ++j, ++i) {
                     if (!wait_bar(&sh.empty[st], ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
                         stop = true;
                         break;
@@ -301,9 +318,8 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     if (sg.kind == 0) {
                         GR_TRACE(kGtLastALoad);
                         const int kbA = (int)(j - sg.first);
-                        mbar_arrive_expect_tx(&sh.full_w[st], kGrWBytes + Cfg::kActBytes);
+                        mbar_arrive_expect_tx(&sh.full_w[st], kGrWBytes);
                         tma_load_2d(w, &tm_win, &sh.full_w[st], kbA * 64, sg.e * a.d_e + sg.mt * 128, pol_weights);
-                        tma_load_2d(w + kGrWBytes, &tm_x, &sh.full_w[st], kbA * 64, sg.g * a.NT, pol_keep);
                     } else {
                         const int e = sh.s_elist[sidx];
                         mbar_arrive_expect_tx(&sh.full_w[st], kGrWBytes);
@@ -385,12 +401,13 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         if (leader) umma_commit(&sh.mma_done);
         __syncwarp();
     } else if (warp == 2) {
-        // ----------------------------------------------------- h' tile loader --
-        // An expert-in stage carries no h': lane 0 just arrives.  For an expert-out
-        // tile, lane 0 waits (bounded) until every contributor of the expert-in
-        // unit holding the tile's 64 columns of h' has written its rows, then moves
-        // the [N x 64] slice by TMA (it lands in the 128-byte-swizzled layout the
-        // MMA reads).
+        // ------------------------------------------------ activation loader --
+        // An expert-in stage's activations are the group's x tile (read once per
+        // expert of the group's set: kept in L2).  For an expert-out tile, lane 0
+        // waits (bounded) until every contributor of the expert-in unit holding
+        // the tile's 64 columns of h' has written its rows, then moves the
+        // [N x 64] slice by TMA (it lands in the 128-byte-swizzled layout the MMA
+        // reads).
         GrIter it;
         it.init(aLo, aHi, bLo, bHi);
         GrSeg sg;
@@ -399,7 +416,7 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         long long i = 0, nB = 0;
         bool stop = sh.abort != 0;
         uint32_t last_u = 0xffffffffu;
-        const uint64_t pol = policy_evict_last();   // an h' tile is read once per row tile of y
+        const uint64_t pol = policy_evict_last();   // x: once per expert; h': once per row tile of y
         if (lane == 0) {
             while (!stop && it.next(a, sg)) {
                 int sidx = 0, kb = 0;
@@ -407,6 +424,11 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     const long long local = sg.lo - sg.first;
                     sidx = (int)(local / a.KBe);
                     kb = (int)(local - (long long)sidx * a.KBe);
+                    if (sg.lo == bLo && aHi > aLo &&
+                        !wait_bar(&sh.a_pub, 0u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
+                        stop = true;
+                        break;
+                    }
                 }
                 for (long long j = sg.lo; j < sg.hi; ++j, ++i) {
                     if (!wait_bar(&sh.empty[st], ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) {
@@ -414,14 +436,15 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                         break;
                     }
                     if (sg.kind == 0) {
-                        mbar_arrive(&sh.full_h[st]);
+                        mbar_arrive_expect_tx(&sh.full_h[st], (uint32_t)Cfg::kActBytes);
+                        tma_load_2d(smem + st * kStageBytes + kGrWBytes, &tm_x, &sh.full_h[st],
+                                    (int)(j - sg.first) * 64, sg.g * a.NT, pol);
                     } else {
                         const int p = sg.off + sidx;
                         const uint32_t u = (uint32_t)(p * a.MT + (kb >> 1));
                         if (u != last_u) {
-                            const long long fA = (long long)u * a.KB;
-                            const int ncA = gr_contributors(fA, fA + a.KB - 1, NA, G, -1).n;
-                            if (!wait_count(&readyA[u], (uint32_t)ncA, limit_peer, &sh.abort, a.ctl)) {
+                            // one block computes the whole expert-in unit and counts it in once
+                            if (!wait_count(&readyA[u], 1u, limit_peer, &sh.abort, a.ctl)) {
                                 stop = true;
                                 break;
                             }
@@ -447,11 +470,9 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 }
             }
             // no copy into this block's shared memory outlives it: the last
-            // kStages stages issued (only B stages carry bytes)
-            if (nB > 0) {
-                for (long long k = i - kStages < 0 ? 0 : i - kStages; k < i; ++k)
-                    wait_bar_drain(&sh.full_h[k % kStages], (uint32_t)((k / kStages) & 1), limit, a.ctl);
-            }
+            // kStages stages issued
+            for (long long k = i - kStages < 0 ? 0 : i - kStages; k < i; ++k)
+                wait_bar_drain(&sh.full_h[k % kStages], (uint32_t)((k / kStages) & 1), limit, a.ctl);
         }
         __syncwarp();
     } else {
@@ -464,10 +485,8 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             // them and has finished; the launch after this one will use them
             const int oth = par ^ 1;
             const long long step = (long long)G * 128;
-            for (long long k = (long long)cta * 128 + et; k < a.cnt_a_len; k += step) {
-                a.cntA[(size_t)oth * a.cnt_a_len + k] = 0u;
+            for (long long k = (long long)cta * 128 + et; k < a.cnt_a_len; k += step)
                 a.readyA[(size_t)oth * a.cnt_a_len + k] = 0u;
-            }
             for (long long k = (long long)cta * 128 + et; k < a.cnt_b_len; k += step)
                 a.cntB[(size_t)oth * a.cnt_b_len + k] = 0u;
         }
@@ -498,101 +517,106 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         // decisions come from shared words read after named barriers
         bool failed = sh.abort0 != 0;   // (the tables are not read after an error)
 
-        // finish the rows [r0, r1) slice of split unit (sg, cb): sum the partials
-        // in block order, then gated Swish + mask into h' (A) or store y (B)
+        // finish the rows [r0, r1) slice of split expert-out unit (sg, cb): sum the
+        // contributors' partial tiles in block order (a fixed order) and store those
+        // rows of y.  Items are (row, token quad); a thread takes 4 items per pass
+        // and, per pass, issues the loads of 4 contributors at once.
         auto finish_split = [&](const GrSeg& sg, const GrContrib& cb) -> bool {
-            const long long total = sg.kind == 0 ? NA : NB;
-            uint32_t* cnt = (sg.kind == 0 ? cntA : cntB) + sg.unit;
+            uint32_t* cnt = cntB + sg.unit;
             if (et == 0) {
                 sh.ep_ok = wait_count(cnt, (uint32_t)cb.n, limit_peer, &sh.abort, a.ctl, kWaitPeers) ? 1 : 0;
                 int k = 0;
                 for (int qq = cb.q0; qq <= cb.q1 && k < kGrMaxContrib; ++qq) {
-                    const long long lo = gr_range_lo(total, G, qq);
-                    if (gr_range_lo(total, G, qq + 1) > lo) sh.s_contrib[k++] = qq * 2 + (lo >= sg.first ? 0 : 1);
+                    const long long lo = gr_range_lo(NB, G, qq);
+                    if (gr_range_lo(NB, G, qq + 1) > lo) sh.s_contrib[k++] = qq * 2 + (lo >= sg.first ? 0 : 1);
                 }
             }
             named_bar_sync(1, 128);
             if (!sh.ep_ok) return false;
-            if (sg.kind == 0) stage_gates(sg.g, sg.e);
-            const float* part = sg.kind == 0 ? a.partA : a.partB;
-            const float4* pbase = reinterpret_cast<const float4*>(part);
+            const float4* pbase = reinterpret_cast<const float4*>(a.partB);
             const int r0 = cb.rank * 128 / cb.n, r1 = (cb.rank + 1) * 128 / cb.n;
             const int nrows = r1 - r0;
             const int nvalid = min(a.NT, a.T - sg.g * a.NT);   // tokens of the group
-            // items (row, token quad) of the slice; per pass every contributor's
-            // float4 is requested before any is used, 8 contributors at a time
             const int nitems = nrows * (N / 4);
-            for (int base = 0; base < nitems; base += 256) {
-                int rr[2], kq[2];
-                bool on[2];
+            for (int base = 0; base < nitems; base += 4 * 128) {
+                int rr[4], kq[4];
+                bool on[4];
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
+                for (int m = 0; m < 4; ++m) {
                     const int itx = base + m * 128 + et;
                     on[m] = itx < nitems;
                     const int ic = on[m] ? itx : 0;
                     rr[m] = r0 + ic % nrows;       // consecutive threads: consecutive rows
                     kq[m] = ic / nrows;            // token quad
                 }
-                float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-                for (int c0 = 0; c0 < cb.n; c0 += 8) {
-                    float4 t4[2][8];
+                float4 acc[4];
 #pragma unroll
-                    for (int m = 0; m < 2; ++m)
+                for (int m = 0; m < 4; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int c0 = 0; c0 < cb.n; c0 += 4) {
+                    float4 t4[4][4];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            t4[m][u] = __ldcg(pbase + (size_t)sh.s_contrib[min(c0 + u, cb.n - 1)] * (N * 32) +
-                                              kq[m] * 128 + rr[m]);
+                    for (int u = 0; u < 4; ++u) {
+                        const float4* src = pbase + (size_t)sh.s_contrib[min(c0 + u, cb.n - 1)] * (N * 32);
 #pragma unroll
-                    for (int m = 0; m < 2; ++m)
+                        for (int m = 0; m < 4; ++m)
+                            t4[u][m] = (c0 + u < cb.n && on[m]) ? __ldcg(src + kq[m] * 128 + rr[m])
+                                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
+                    for (int u = 0; u < 4; ++u)
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
                             if (c0 + u < cb.n) {
-                                acc[m].x += t4[m][u].x;
-                                acc[m].y += t4[m][u].y;
-                                acc[m].z += t4[m][u].z;
-                                acc[m].w += t4[m][u].w;
+                                acc[m].x += t4[u][m].x;
+                                acc[m].y += t4[u][m].y;
+                                acc[m].z += t4[u][m].z;
+                                acc[m].w += t4[u][m].w;
                             }
                         }
                 }
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
+                for (int m = 0; m < 4; ++m) {
                     if (!on[m]) continue;
                     const float z[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
-                    if (sg.kind == 0) {
-                        __nv_bfloat16* hrow = a.hbuf + (size_t)sg.p * N * a.d_e + sg.mt * 128 + rr[m];
+                    __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + rr[m];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int j = 4 * kq[m] + u;
-                            const bool bit = (sh.s_bits[j >> 5] >> (j & 31)) & 1u;
-                            const float h = bit ? sh.s_gv[j] * gr_swish(z[u]) : 0.f;
-                            hrow[(size_t)j * a.d_e] = __float2bfloat16_rn(h);
-                        }
-                    } else {
-                        __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + rr[m];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int j = 4 * kq[m] + u;
-                            if (j < nvalid) ycol[(size_t)j * a.d_h] = __float2bfloat16_rn(z[u]);
-                        }
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = 4 * kq[m] + u;
+                        if (j < nvalid) ycol[(size_t)j * a.d_h] = __float2bfloat16_rn(z[u]);
                     }
                 }
             }
-            // every thread is done with sh.ep_ok and (A) the staged gates before the
-            // next unit's wait rewrites them
+            // every thread is done with sh.ep_ok before the next unit's wait rewrites it
             named_bar_sync(1, 128);
             return true;
         };
-        // this block's rows of h' for expert-in unit `unit` are written: count it in
-        auto announce_ready = [&](uint32_t unit) {
-            __threadfence();
+        // Announcements.  A release waits for the block's bulk copies in flight, so
+        // the block announces in two batches, each when none of its copies is in
+        // flight: all its expert-in units once the last one's h' is written (the
+        // producer and the loader hold their first expert-out copy until then), and
+        // all its expert-out partials after its last accumulator.  One thread fences
+        // after a barrier that orders every thread's stores before it.
+        const long long uLo = aLo / a.KB, uHi = aHi / a.KB;   // this block's expert-in units
+        auto announce_a = [&]() {
             named_bar_sync(1, 128);
-            if (et == 0 && (int)unit != a.skip_flag_unit) atomicAdd(&readyA[unit], 1u);
+            if (et == 0) {
+                GR_TRACE(kGtAnnounce);
+                __threadfence();
+                for (long long u = uLo; u < uHi; ++u)
+                    if ((int)u != a.skip_flag_unit) atomicAdd(&readyA[u], 1u);
+                mbar_arrive(&sh.a_pub);
+                GR_TRACE(kGtAFlushed);
+            }
         };
         auto flush_pending = [&]() -> bool {
-            for (int k = 0; k < npend; ++k) {
-                if (!finish_split(pend_sg[k], pend_cb[k])) return false;
-                if (pend_sg[k].kind == 0) announce_ready(pend_sg[k].unit);
+            if (npend == 0) return true;
+            named_bar_sync(1, 128);
+            if (et == 0) {
+                __threadfence();
+                for (int k = 0; k < npend; ++k) atomicAdd(cntB + pend_sg[k].unit, 1u);
             }
+            for (int k = 0; k < npend; ++k)
+                if (!finish_split(pend_sg[k], pend_cb[k])) return false;
             npend = 0;
             return true;
         };
@@ -604,12 +628,17 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         int cur_kind = 0;
         while (!failed && it.next(a, sg)) {
             if (sg.kind != cur_kind) {
-                if (!flush_pending()) { failed = true; break; }
+                if (uHi > uLo) announce_a();
                 cur_kind = sg.kind;
-                if (et == 0) GR_TRACE(kGtAFlushed);
             }
-            const long long total = sg.kind == 0 ? NA : NB;
-            const GrContrib cb = gr_contributors(sg.first, sg.last, total, G, cta);
+            GrContrib cb;
+            if (sg.kind == 0) {
+                cb.q0 = cb.q1 = cta;   // whole expert-in units: never split
+                cb.n = 1;
+                cb.rank = 0;
+            } else {
+                cb = gr_contributors(sg.first, sg.last, NB, G, cta);
+            }
             // stage this unit's gates while its accumulator completes
             if (sg.kind == 0 && cb.n == 1) stage_gates(sg.g, sg.e);
             const int ab = (int)(acc_i & 1u);
@@ -626,46 +655,65 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * N);
             const int nvalid = min(a.NT, a.T - sg.g * a.NT);   // tokens of the group
             if (cb.n == 1) {
-                // the whole unit is here: all 128 rows straight from the accumulator
+                // The whole unit is here: all 128 rows straight from the accumulator,
+                // 32 tokens at a time.  Each slice is staged token-major in shared
+                // memory ([32 tokens][128 rows] bf16: a token's 128 rows are 256
+                // contiguous bytes of h' or y) and written with 16-byte stores.
+                __nv_bfloat16* dst;
+                size_t ld;
+                int ntok;
                 if (sg.kind == 0) {
-                    __nv_bfloat16* hrow = a.hbuf + (size_t)sg.p * N * a.d_e + sg.mt * 128 + row;
+                    dst = a.hbuf + (size_t)sg.p * N * a.d_e + sg.mt * 128;
+                    ld = (size_t)a.d_e;
+                    ntok = N;                      // h' rows of every token (masked ones are 0)
+                } else {
+                    dst = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128;
+                    ld = (size_t)a.d_h;
+                    ntok = nvalid;
+                }
 #pragma unroll 1
-                    for (int c0 = 0; c0 < N; c0 += 32) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
-                        tmem_ld_wait();
+                for (int c0 = 0; c0 < N; c0 += 32) {
+                    __nv_bfloat16* stg = ostage + ((c0 >> 5) & 1) * (32 * 128);
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
+                    tmem_ld_wait();
+                    if (sg.kind == 0) {
                         const uint32_t bits = sh.s_bits[c0 >> 5];
 #pragma unroll
                         for (int u = 0; u < 32; ++u) {
                             const float h = ((bits >> u) & 1u) ? sh.s_gv[c0 + u] * gr_swish(__uint_as_float(r[u])) : 0.f;
-                            hrow[(size_t)(c0 + u) * a.d_e] = __float2bfloat16_rn(h);
+                            stg[u * 128 + row] = __float2bfloat16_rn(h);
                         }
-                    }
-                } else {
-                    __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + row;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < N; c0 += 32) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
-                        tmem_ld_wait();
+                    } else {
 #pragma unroll
-                        for (int u = 0; u < 32; ++u)
-                            if (c0 + u < nvalid) ycol[(size_t)(c0 + u) * a.d_h] = __float2bfloat16_rn(__uint_as_float(r[u]));
+                        for (int u = 0; u < 32; ++u) stg[u * 128 + row] = __float2bfloat16_rn(__uint_as_float(r[u]));
+                    }
+                    named_bar_sync(1, 128);
+                    if (et == 0 && acc_i == 0 && c0 == 0) GR_TRACE(kGtFirstSlice);
+                    // 32 tokens x 16 pieces of 16 bytes; (the other staging slice is
+                    // being filled meanwhile, so one barrier per slice suffices)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int c = et + 128 * k;
+                        const int tok = c >> 4, piece = c & 15;
+                        if (c0 + tok < ntok)
+                            *reinterpret_cast<uint4*>(dst + (size_t)(c0 + tok) * ld + piece * 8) =
+                                reinterpret_cast<const uint4*>(stg + tok * 128)[piece];
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.acc_empty[ab]);
+                if (et == 0 && acc_i == 0) GR_TRACE(kGtADrained);
                 ++acc_i;
-                if (sg.kind == 0) announce_ready(sg.unit);   // also frees the staged gates
+                if (sg.kind == 0) named_bar_sync(1, 128);   // the staged gates are free again
             } else {
                 // publish this block's partial tile and count it in; the slice is
                 // finished in the second pass.  Layout: float4 (token quad k, row)
                 // at k * 128 + row.
-                float* part = sg.kind == 0 ? a.partA : a.partB;
-                uint32_t* cnt = (sg.kind == 0 ? cntA : cntB) + sg.unit;
-                const long long myLo = sg.kind == 0 ? aLo : bLo;
-                const int myslot = myLo >= sg.first ? 0 : 1;
+                // (only expert-out units are ever split)
+                float* part = a.partB;
+                const int myslot = bLo >= sg.first ? 0 : 1;
                 float4* dst = reinterpret_cast<float4*>(part + (size_t)(cta * 2 + myslot) * (N * 128)) + row;
 #pragma unroll 1
                 for (int c0 = 0; c0 < N; c0 += 32) {
@@ -682,9 +730,6 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.acc_empty[ab]);
                 ++acc_i;
-                __threadfence();
-                named_bar_sync(1, 128);
-                if (et == 0) atomicAdd(cnt, 1u);
                 if (npend < 2) {
                     pend_sg[npend] = sg;
                     pend_cb[npend] = cb;
@@ -692,6 +737,7 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 }
             }
         }
+        if (!failed && cur_kind == 0 && uHi > uLo) announce_a();   // expert-in work only
         if (!failed) flush_pending();
         if (et == 0) GR_TRACE(kGtEpiEnd);
     }
@@ -704,20 +750,13 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const uint32_t old = atomicAdd(&a.ctl->done, 1u);
-        if (old == (uint32_t)(G - 1)) {
-            a.ctl->done = 0u;
-            atomicExch(&a.ctl->epoch, stamp);
-        }
-        GR_TRACE(kGtEnd);
-    }
+    if (threadIdx.x == 0) GR_TRACE(kGtEnd);
 }
 
 template <int N>
 static size_t group_smem_bytes() {
-    return 1024 + (size_t)GrCfg<N>::kStages * GrCfg<N>::kStageBytes + sizeof(GrShared<N>);
+    return 1024 + (size_t)GrCfg<N>::kStages * GrCfg<N>::kStageBytes + sizeof(GrShared<N>) + 1024 +
+           kGrOutStageBytes;
 }
 
 template <int N>

@@ -53,10 +53,8 @@ struct GrArgs {
     const int32_t* goffsets;  // [NGr + 1]
     const int32_t* gpair;     // [P] (group << 8) | expert, by group, experts ascending
     __nv_bfloat16* hbuf;      // [P][N][d_e] gated activations h'
-    float* partA;             // [grid][2][N*128] split-K partial sums (expert-in)
     float* partB;             // [grid][2][N*128] split-expert partial sums (expert-out)
-    uint32_t* cntA;           // [2][cnt_a_len] blocks that published an expert-in partial
-    uint32_t* readyA;         // [2][cnt_a_len] blocks whose rows of h' are written
+    uint32_t* readyA;         // [2][cnt_a_len] expert-in units whose h' is written
     uint32_t* cntB;           // [2][cnt_b_len] blocks that published an expert-out partial
     long long cnt_a_len;      // NGr*E*MT
     long long cnt_b_len;      // NGr*RT
