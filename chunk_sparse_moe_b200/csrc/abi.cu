@@ -103,6 +103,20 @@ bool make_map_kpair(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
     return map_kblocks(m, base, cols, rows, box_rows, 2);
 }
 
+// 2-D fp32 tensor [outer, inner], box {box_inner, box_outer}, no swizzle.
+bool make_map_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 4};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor [outer, inner], box {box_inner, box_outer}, no swizzle (for
 // tiled stores from a plain row-major shared-memory tile).
 bool make_map_plain(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -434,11 +448,14 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     e = launch_group_plan(g, T, E, n, t_counts, t_idx, t_tmask, !tables, ctl, L.NG, L.NGr, gcounts, goffsets,
                           gpair, static_cast<__nv_bfloat16*>(y), d_h, s);
     if (e != cudaSuccess) return cuda_fail(e, "group plan launch");
-    CUtensorMap maps[4];
+    CUtensorMap maps[5];
+    // expert-out partial tiles [blocks][2 slots][N/4 token quads][128 rows x 4 tokens]
+    // fp32, seen as lines of 512 floats; a box is 32 rows of every token quad
     if (!make_map(&maps[0], x, (uint64_t)d_h, (uint64_t)T, (uint32_t)L.N) ||
         !make_map(&maps[1], W_in, (uint64_t)d_h, (uint64_t)E * d_e, 128) ||
         !make_map(&maps[2], W_out, (uint64_t)d_e, (uint64_t)E * d_h, 128) ||
-        !make_map(&maps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)L.Pmax * L.N, (uint32_t)L.N))
+        !make_map(&maps[3], ws + L.hbuf, (uint64_t)d_e, (uint64_t)L.Pmax * L.N, (uint32_t)L.N) ||
+        !make_map_f32(&maps[4], ws + L.partB, 512, (uint64_t)G * 2 * (L.N / 4), 128, (uint32_t)(L.N / 4)))
         return fail(BLOCKFFN_ERR_CUDA, "cuTensorMapEncodeTiled failed");
     GrArgs a;
     a.gates = g;

@@ -39,7 +39,8 @@ enum : int32_t {
 struct Ctl {
     int32_t status;        // first device-side error (sticky until reset)
     int32_t detail;        // which wait / check
-    uint32_t unused_[2];
+    uint32_t plan_done;    // blocks of the current group-plan launch that finished (the last resets it)
+    uint32_t unused_;
     uint32_t issued[2];    // by launch parity: blocks that issued their last expert-in load
     // The shapes, dtype, gating mode and kernel the workspace's layout was made
     // for, claimed by the first launch after a reset (0 = not yet bound).  A

@@ -27,7 +27,7 @@
 // Expert-out (B).  y^T = sum_e W_out_e h'_e^T with W_out_e's 128-row tiles as the
 // M operand and the tokens as N.  Cluster c owns the row tiles c, c + #clusters,
 // ...; each of its 4 blocks takes a quarter of a row tile's (expert, pair of
-// 64-wide k-blocks) tiles.  A tile waits (bounded) until every expert's h' is counted
+// 64-wide k-blocks) tiles.  A tile waits (bounded) until its expert's h' is counted
 // in, then its h' slice arrives by TMA.  The 4 partial tiles are summed inside
 // the cluster: warp q of every block st.async's its 32 accumulator rows to the
 // block of rank q, which adds the 4 contributions in rank order (a fixed order)
@@ -536,10 +536,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // An expert-in stage's activations are the chunk's two x k-blocks of the
         // stage (lane 0 issues them, so the weight tiles and the activation tiles
         // come from two issuing threads: one thread issues bulk copies at a bounded
-        // rate).  Before the first expert-out tile the warp waits (bounded) until
-        // every expert slot's h' is counted in; then lane 0 moves each tile's
-        // [N x 64] h' slice with one TMA load, which lands in the same
-        // 128-byte-swizzled layout as the weight tile's operand.
+        // rate).  For an expert-out tile lane 0 waits (bounded) until the tile's
+        // expert slot's h' is counted in, then moves the [N x 64] h' slice with
+        // one TMA load, which lands in the same 128-byte-swizzled layout as the
+        // weight tile's operand.
         long long i = 0;
         RingPos rp;
         int stop = sh.abort != 0;
@@ -558,49 +558,31 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
         }
         stop = __shfl_sync(0xffffffffu, stop, 0);
-        if (!stop && totB > 0) {
-            // The expert-in units all finish at about the same time, so one combined
-            // wait costs no more than the slowest slot; each poll round checks 32
-            // slots at once (one acquire load per lane).
-            const uint64_t t0 = globaltimer_ns();
-            bool done = false;
-            while (!done) {
-                bool mine_ok = true;
-                for (int q = lane; q < P; q += 32)
-                    if (ld_acquire_gpu(&readyA[q]) < (uint32_t)(2 * MT)) mine_ok = false;
-                done = __all_sync(0xffffffffu, mine_ok);
-                if (done) break;
-                __nanosleep(64);
-                // the whole warp gives up together: lane 0's clock decides the
-                // timeout (lanes read the clock at slightly different times)
-                const bool aborted = __any_sync(0xffffffffu, sh.abort != 0);
-                const bool timed_out = __shfl_sync(0xffffffffu, globaltimer_ns() - t0 > limit_peer ? 1 : 0, 0) != 0;
-                if (aborted || timed_out) {
-                    if (lane == 0 && !aborted) {
-                        record_error(a.ctl, kErrTimeout, kWaitFlag);
-                        sh.abort = 1;
-                    }
-                    break;
+        if (!stop && totB > 0 && lane == 0) {
+            // Each expert-out tile waits (bounded) only for its own expert slot's h'
+            // (both k-halves of every 128-row tile counted in), so tiles of experts
+            // finished early start while later experts' expert-in units still run.
+            const uint64_t pol = policy_evict_first();
+            BCursor bc;
+            bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
+            int ready_s = -1;
+            for (int q = 0; q < totB; ++q, ++i, rp.advance(), bc.advance()) {
+                if (bc.s != ready_s) {
+                    if (!wait_count(&readyA[bc.s], (uint32_t)(2 * MT), limit_peer, &sh.abort, a.ctl)) break;
+                    // the h' stores were made visible to this thread by the acquire;
+                    // the async proxy reads them next
+                    fence_proxy_async_global();
+                    if (ready_s < 0) RS_TRACE_ONCE(kRtFirstFlag);
+                    RS_TRACE(kRtLastFlag);
+                    ready_s = bc.s;
                 }
-            }
-            __syncwarp();
-            if (lane == 0 && done) {
-                // the h' stores were made visible to this thread by the acquires; the
-                // async proxy reads them next
-                fence_proxy_async_global();
-                RS_TRACE_ONCE(kRtFirstFlag);
-                RS_TRACE(kRtLastFlag);
-                const uint64_t pol = policy_evict_first();
-                BCursor bc;
-                bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
-                for (int q = 0; q < totB; ++q, ++i, rp.advance(), bc.advance()) {
-                    if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) break;
-                    mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 256));
-                    tma_load_3d(smem + rp.st * kRsStageBytes + kRsWBytes, &tm_h, &sh.full_h[rp.st], 0, bc.s * N,
-                                2 * bc.kb, pol);
-                }
+                if (!wait_bar(&sh.empty[rp.st], rp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) break;
+                mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 256));
+                tma_load_3d(smem + rp.st * kRsStageBytes + kRsWBytes, &tm_h, &sh.full_h[rp.st], 0, bc.s * N,
+                            2 * bc.kb, pol);
             }
         }
+        __syncwarp();
         if (lane == 0) {
             // no copy into this block's shared memory outlives it: the last ring's
             // worth of stages this warp filled (x or h'; an earlier stage's slot was
@@ -714,12 +696,18 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             // its h is not finite), staged token-major in shared memory, then written
             // with 16-byte stores: token t's 128 rows are 256 contiguous bytes
             {
+                // gates into registers first (loads interleaved with the staging
+                // stores would each wait for the store before them)
+                float gv[NH];
+#pragma unroll
+                for (int tl = 0; tl < NH; ++tl) gv[tl] = sh.s_gate[b][tg + tl];
+                __nv_bfloat16 hb[NH];
+#pragma unroll
+                for (int tl = 0; tl < NH; ++tl)
+                    hb[tl] = __float2bfloat16_rn(((bits >> tl) & 1u) ? gv[tl] * rs_swish(z[tl]) : 0.f);
                 __nv_bfloat16* stg = hstage + row;
 #pragma unroll
-                for (int tl = 0; tl < NH; ++tl) {
-                    const float gsw = sh.s_gate[b][tg + tl] * rs_swish(z[tl]);
-                    stg[tl * 128] = __float2bfloat16_rn(((bits >> tl) & 1u) ? gsw : 0.f);
-                }
+                for (int tl = 0; tl < NH; ++tl) stg[tl * 128] = hb[tl];
             }
             named_bar_sync(1, 128);
             {

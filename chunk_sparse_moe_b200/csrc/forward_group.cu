@@ -50,12 +50,14 @@ namespace bffn {
 
 namespace {
 
-constexpr int kGrThreads = 224;
+constexpr int kGrThreads = 352;               // 3 role warps + 8 epilogue warps
+constexpr int kGrEpi = 256;                    // epilogue threads
 constexpr int kGrWBytes = 128 * 128;            // weight tile: 128 rows x 64 bf16
 constexpr int kGrMaxE = 256;
 constexpr int kGrMaxContrib = 160;              // >= blocks per launch (one per SM)
 constexpr int kGrSmemBudget = 200 * 1024;       // pipeline stages
-// epilogue output staging: two [32 tokens][128 rows] bf16 slices (8 KB each)
+// epilogue output staging: one [32 tokens][128 rows] bf16 slice (8 KB) per
+// epilogue warp group
 constexpr int kGrOutStageBytes = 2 * 32 * 128 * 2;
 
 template <int N>
@@ -75,6 +77,7 @@ struct GrShared {
     uint64_t acc_empty[2];
     uint64_t mma_done;
     uint64_t a_pub;                        // this block's expert-in results are announced
+    uint64_t flush_bar;                    // partial tiles landed in the idle ring (TMA bytes)
     uint32_t tmem_base;
     volatile int abort;
     int abort0;                            // abort as set before the first block barrier
@@ -83,7 +86,7 @@ struct GrShared {
     int ep_ok;
     int s_contrib[kGrMaxContrib];
     int32_t s_elist[kGrMaxE];              // producer: experts of the current B unit
-    float s_gv[N];                         // epilogue: the unit's gates (0 where masked)
+    alignas(16) float s_gv[N];             // epilogue: the unit's gates (0 where masked)
     uint32_t s_bits[N / 32];               // epilogue: the unit's token bits
 };
 
@@ -195,7 +198,10 @@ enum : int {
     kGtStart = 0, kGtPrologue = 1, kGtFirstLoad = 2, kGtLastALoad = 3, kGtLastACommit = 4,
     kGtAFlushed = 5, kGtFirstFlag = 6, kGtLastBCommit = 7, kGtEpiEnd = 8, kGtEnd = 9,
     kGtFirstAcc = 10, kGtFirstBLoad = 11, kGtLastLoad = 12, kGtADrained = 13, kGtAnnounce = 14,
-    kGtFirstSlice = 15, kGtSlots = 64
+    kGtFirstSlice = 15, kGtSliceBase = 16,   // 16 + 4*slice + step, first unit only (steps: TMEM read,
+                                             // staged, barrier passed, stores issued)
+    kGtLoopEnd = 48, kGtFlushAnnounced = 49, kGtFinBase = 50,   // 50 + 3*k + {counted, copied, summed}
+    kGtSlots = 64
 };
 #define GR_TRACE(slot) \
     do { if (a.trace) a.trace[(size_t)blockIdx.x * kGtSlots + (slot)] = globaltimer_ns(); } while (0)
@@ -206,7 +212,7 @@ template <int N>
 __global__ void __launch_bounds__(kGrThreads, 1)
 union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_win,
                    const __grid_constant__ CUtensorMap tm_wout, const __grid_constant__ CUtensorMap tm_h,
-                   const GrArgs a) {
+                   const __grid_constant__ CUtensorMap tm_part, const GrArgs a) {
     using Cfg = GrCfg<N>;
     constexpr int kStages = Cfg::kStages;
     constexpr int kStageBytes = Cfg::kStageBytes;
@@ -219,6 +225,10 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, cta = blockIdx.x;
 
+    // Set-up that touches only this block's shared memory, TMEM and the tensor
+    // maps runs first; the kernel is a programmatic dependent of the group-plan
+    // kernel and waits for it (griddepcontrol.wait) before reading the control
+    // block, the tables or any input.
     if (threadIdx.x == 0) {
         GR_TRACE(kGtStart);
         for (int s = 0; s < kStages; ++s) {
@@ -228,12 +238,25 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sh.acc_full[s], 1);
-            mbar_init(&sh.acc_empty[s], 4);
+            mbar_init(&sh.acc_empty[s], 8);   // one arrival per epilogue warp
         }
         mbar_init(&sh.mma_done, 1);
         mbar_init(&sh.a_pub, 1);
+        mbar_init(&sh.flush_bar, 1);
         fence_mbar_init();
-        // written by earlier launches only: plain L2 loads
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_win);
+        prefetch_tmap(&tm_wout);
+        prefetch_tmap(&tm_h);
+        prefetch_tmap(&tm_part);
+    }
+    if (warp == 2) {
+        tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    griddep_wait();
+    if (threadIdx.x == 0) {
+        griddep_launch_dependents();
         const int32_t st0 = __ldcg(&a.ctl->status);
         const unsigned long long tk = atomicAdd(&a.ctl->ticket, 1ull);   // launch index = ticket / grid
         const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
@@ -243,14 +266,6 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         sh.abort = st0 != 0 || !key_ok;
         sh.abort0 = st0 != 0 || !key_ok;
         sh.epoch = ep0;
-        prefetch_tmap(&tm_x);
-        prefetch_tmap(&tm_win);
-        prefetch_tmap(&tm_wout);
-        prefetch_tmap(&tm_h);
-    }
-    if (warp == 2) {
-        tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -476,25 +491,31 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         }
         __syncwarp();
     } else {
-        // --------------------------------------------------- epilogue (3-6) --
+        // ------------------------------------------------ epilogue (warps 3-10) --
+        // Eight warps: two per TMEM lane quadrant (a warp reads the quadrant of its
+        // index modulo 4).  Warp group eg (warps 3-6: 0, warps 7-10: 1) drains the
+        // accumulator's 32-column slices eg, eg + 2, ...; named barrier 1 joins all
+        // 256 threads, barrier 2 + eg the 128 threads of one group.
         const int q = warp & 3;
         const int row = q * 32 + lane;           // accumulator row = TMEM lane
-        const int et = threadIdx.x - 96;         // 0..127
+        const int et = threadIdx.x - 96;         // 0..255
+        const int eg = et >> 7;                  // warp group
+        const int gt = et & 127;                 // thread within the group
         {
             // zero the other parity's counters: the launch before this one used
             // them and has finished; the launch after this one will use them
             const int oth = par ^ 1;
-            const long long step = (long long)G * 128;
-            for (long long k = (long long)cta * 128 + et; k < a.cnt_a_len; k += step)
+            const long long step = (long long)G * kGrEpi;
+            for (long long k = (long long)cta * kGrEpi + et; k < a.cnt_a_len; k += step)
                 a.readyA[(size_t)oth * a.cnt_a_len + k] = 0u;
-            for (long long k = (long long)cta * 128 + et; k < a.cnt_b_len; k += step)
+            for (long long k = (long long)cta * kGrEpi + et; k < a.cnt_b_len; k += step)
                 a.cntB[(size_t)oth * a.cnt_b_len + k] = 0u;
         }
         // the gates of expert e for the tokens of group g, zero where the token's
         // bit in its chunk's mask is clear or the token lies past the group or T,
-        // and the bits themselves; staged in shared memory by the 128 threads
+        // and the bits themselves; staged in shared memory by the 256 threads
         auto stage_gates = [&](int g, int e) {
-            for (int j = et; j < N; j += 128) {
+            for (int j = et; j < N; j += kGrEpi) {
                 const int t = g * a.NT + j;
                 bool bit = false;
                 float gv = 0.f;
@@ -507,89 +528,99 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 const uint32_t bal = __ballot_sync(0xffffffffu, bit);
                 if (lane == 0) sh.s_bits[j >> 5] = bal;
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kGrEpi);
         };
 
-        GrSeg pend_sg[2];
-        GrContrib pend_cb[2];
+        // at most two split expert-out units per block (its first and its last),
+        // kept in fixed slots (no dynamically indexed local array)
+        GrSeg pend_sg[2] = {};
+        GrContrib pend_cb[2] = {};
         int npend = 0;
         // the same in every epilogue thread (fixed before the first barrier); later
         // decisions come from shared words read after named barriers
         bool failed = sh.abort0 != 0;   // (the tables are not read after an error)
+        uint32_t flush_phase = 0u;
 
-        // finish the rows [r0, r1) slice of split expert-out unit (sg, cb): sum the
+        // Finish the rows [r0, r1) slice of split expert-out unit (sg, cb): sum the
         // contributors' partial tiles in block order (a fixed order) and store those
-        // rows of y.  Items are (row, token quad); a thread takes 4 items per pass
-        // and, per pass, issues the loads of 4 contributors at once.
-        auto finish_split = [&](const GrSeg& sg, const GrContrib& cb) -> bool {
+        // rows of y.  This runs after the block's last accumulator, when the stage
+        // ring is idle: the contributors' rows come by TMA, one box of 32 rows x N
+        // tokens per (contributor, 32 rows), as many at a time as the ring holds
+        // beside a running-sum region, and are added in shared memory.  The loops
+        // are kept rolled: this code runs once per launch, so its size (fetched
+        // cold) costs more than its loop overhead.
+        constexpr int kBoxF4 = 32 * (N / 4);                // float4 per box: 32 rows x N tokens
+        constexpr int kBoxBytes = kBoxF4 * 16;
+        constexpr int kRingBoxes = kStages * kStageBytes / kBoxBytes;
+        auto finish_split = [&](const GrSeg& sg, const GrContrib& cb, int kslot) -> bool {
             uint32_t* cnt = cntB + sg.unit;
             if (et == 0) {
                 sh.ep_ok = wait_count(cnt, (uint32_t)cb.n, limit_peer, &sh.abort, a.ctl, kWaitPeers) ? 1 : 0;
+                GR_TRACE(kGtFinBase + 3 * kslot);
                 int k = 0;
                 for (int qq = cb.q0; qq <= cb.q1 && k < kGrMaxContrib; ++qq) {
                     const long long lo = gr_range_lo(NB, G, qq);
                     if (gr_range_lo(NB, G, qq + 1) > lo) sh.s_contrib[k++] = qq * 2 + (lo >= sg.first ? 0 : 1);
                 }
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kGrEpi);
             if (!sh.ep_ok) return false;
-            const float4* pbase = reinterpret_cast<const float4*>(a.partB);
             const int r0 = cb.rank * 128 / cb.n, r1 = (cb.rank + 1) * 128 / cb.n;
-            const int nrows = r1 - r0;
+            const int nrows = r1 - r0;                        // <= 64
+            const int nb = (nrows + 31) / 32;                 // boxes per contributor
+            const int cap = kRingBoxes / nb - 1;              // contributors per batch
+            const int nitems = nrows * (N / 4);               // (row, token quad) items
+            float4* ring4 = reinterpret_cast<float4*>(smem);  // boxes [0, nb): running sums
             const int nvalid = min(a.NT, a.T - sg.g * a.NT);   // tokens of the group
-            const int nitems = nrows * (N / 4);
-            for (int base = 0; base < nitems; base += 4 * 128) {
-                int rr[4], kq[4];
-                bool on[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int itx = base + m * 128 + et;
-                    on[m] = itx < nitems;
-                    const int ic = on[m] ? itx : 0;
-                    rr[m] = r0 + ic % nrows;       // consecutive threads: consecutive rows
-                    kq[m] = ic / nrows;            // token quad
+            for (int c0 = 0; c0 < cb.n; c0 += cap) {
+                const int cn = min(cap, cb.n - c0);
+                const bool last = c0 + cn == cb.n;
+                if (et == 0) {
+                    // the boxes about to be overwritten were last read by generic loads
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(&sh.flush_bar, (uint32_t)(cn * nb * kBoxBytes));
+                    const uint64_t pol = policy_evict_first();
+#pragma unroll 1
+                    for (int c = 0; c < cn; ++c)
+#pragma unroll 1
+                        for (int b = 0; b < nb; ++b)
+                            tma_load_2d(smem + (size_t)((1 + c) * nb + b) * kBoxBytes, &tm_part, &sh.flush_bar,
+                                        (r0 + 32 * b) * 4, sh.s_contrib[c0 + c] * (N / 4), pol);
+                    sh.ep_ok = wait_bar_drain(&sh.flush_bar, flush_phase, limit, a.ctl) ? 1 : 0;
                 }
-                float4 acc[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int c0 = 0; c0 < cb.n; c0 += 4) {
-                    float4 t4[4][4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float4* src = pbase + (size_t)sh.s_contrib[min(c0 + u, cb.n - 1)] * (N * 32);
-#pragma unroll
-                        for (int m = 0; m < 4; ++m)
-                            t4[u][m] = (c0 + u < cb.n && on[m]) ? __ldcg(src + kq[m] * 128 + rr[m])
-                                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                flush_phase ^= 1u;
+                named_bar_sync(1, kGrEpi);
+                if (!sh.ep_ok) return false;
+#pragma unroll 1
+                for (int i = et; i < nitems; i += kGrEpi) {
+                    const int kq = i / nrows, rr = i - kq * nrows;
+                    const int off = (rr >> 5) * kBoxF4 + kq * 32 + (rr & 31);
+                    float4 acc = c0 == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ring4[off];
+#pragma unroll 1
+                    for (int c = 0; c < cn; ++c) {
+                        const float4 v = ring4[(1 + c) * nb * kBoxF4 + off];
+                        acc.x += v.x;
+                        acc.y += v.y;
+                        acc.z += v.z;
+                        acc.w += v.w;
                     }
+                    if (!last) {
+                        ring4[off] = acc;
+                    } else {
+                        __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + r0 + rr;
+                        const float z[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            if (c0 + u < cb.n) {
-                                acc[m].x += t4[u][m].x;
-                                acc[m].y += t4[u][m].y;
-                                acc[m].z += t4[u][m].z;
-                                acc[m].w += t4[u][m].w;
-                            }
-                        }
-                }
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    if (!on[m]) continue;
-                    const float z[4] = {acc[m].x, acc[m].y, acc[m].z, acc[m].w};
-                    __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + rr[m];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = 4 * kq[m] + u;
-                        if (j < nvalid) ycol[(size_t)j * a.d_h] = __float2bfloat16_rn(z[u]);
+                        for (int u = 0; u < 4; ++u)
+                            if (4 * kq + u < nvalid) ycol[(size_t)(4 * kq + u) * a.d_h] = __float2bfloat16_rn(z[u]);
                     }
                 }
+                named_bar_sync(1, kGrEpi);   // the ring is read; the next batch may land
+                if (et == 0) GR_TRACE(kGtFinBase + 3 * kslot + 1);
             }
-            // every thread is done with sh.ep_ok before the next unit's wait rewrites it
-            named_bar_sync(1, 128);
+            if (et == 0) GR_TRACE(kGtFinBase + 3 * kslot + 2);
             return true;
         };
+
         // Announcements.  A release waits for the block's bulk copies in flight, so
         // the block announces in two batches, each when none of its copies is in
         // flight: all its expert-in units once the last one's h' is written (the
@@ -598,7 +629,7 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         // after a barrier that orders every thread's stores before it.
         const long long uLo = aLo / a.KB, uHi = aHi / a.KB;   // this block's expert-in units
         auto announce_a = [&]() {
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kGrEpi);
             if (et == 0) {
                 GR_TRACE(kGtAnnounce);
                 __threadfence();
@@ -610,13 +641,16 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         };
         auto flush_pending = [&]() -> bool {
             if (npend == 0) return true;
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kGrEpi);
             if (et == 0) {
+                GR_TRACE(kGtLoopEnd);
                 __threadfence();
-                for (int k = 0; k < npend; ++k) atomicAdd(cntB + pend_sg[k].unit, 1u);
+                if (npend >= 1) atomicAdd(cntB + pend_sg[0].unit, 1u);
+                if (npend >= 2) atomicAdd(cntB + pend_sg[1].unit, 1u);
+                GR_TRACE(kGtFlushAnnounced);
             }
-            for (int k = 0; k < npend; ++k)
-                if (!finish_split(pend_sg[k], pend_cb[k])) return false;
+            if (npend >= 1 && !finish_split(pend_sg[0], pend_cb[0], 0)) return false;
+            if (npend >= 2 && !finish_split(pend_sg[1], pend_cb[1], 1)) return false;
             npend = 0;
             return true;
         };
@@ -626,6 +660,7 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         GrSeg sg;
         uint32_t acc_i = 0;
         int cur_kind = 0;
+        __nv_bfloat16* const stg = ostage + eg * (32 * 128);   // this group's staging slice
         while (!failed && it.next(a, sg)) {
             if (sg.kind != cur_kind) {
                 if (uHi > uLo) announce_a();
@@ -643,12 +678,12 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             if (sg.kind == 0 && cb.n == 1) stage_gates(sg.g, sg.e);
             const int ab = (int)(acc_i & 1u);
             const uint32_t aph = (acc_i >> 1) & 1u;
-            // one thread waits and the 128 threads take its decision together, so
+            // one thread waits and the 256 threads take its decision together, so
             // the named barriers below always see all of them
             if (et == 0)
                 sh.ep_wait[acc_i & 1u] =
                     wait_bar(&sh.acc_full[ab], aph, limit, &sh.abort, a.ctl, kWaitAccFull) ? 1 : 0;
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kGrEpi);
             if (!sh.ep_wait[acc_i & 1u]) { failed = true; break; }
             tc_fence_after();
             if (et == 0 && acc_i == 0) GR_TRACE(kGtFirstAcc);
@@ -656,9 +691,10 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             const int nvalid = min(a.NT, a.T - sg.g * a.NT);   // tokens of the group
             if (cb.n == 1) {
                 // The whole unit is here: all 128 rows straight from the accumulator,
-                // 32 tokens at a time.  Each slice is staged token-major in shared
-                // memory ([32 tokens][128 rows] bf16: a token's 128 rows are 256
-                // contiguous bytes of h' or y) and written with 16-byte stores.
+                // 32 tokens at a time, each group its own slices.  A slice is staged
+                // token-major in shared memory ([32 tokens][128 rows] bf16: a token's
+                // 128 rows are 256 contiguous bytes of h' or y) and written with
+                // 16-byte stores.
                 __nv_bfloat16* dst;
                 size_t ld;
                 int ntok;
@@ -672,51 +708,71 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     ntok = nvalid;
                 }
 #pragma unroll 1
-                for (int c0 = 0; c0 < N; c0 += 32) {
-                    __nv_bfloat16* stg = ostage + ((c0 >> 5) & 1) * (32 * 128);
+                for (int c0 = 32 * eg; c0 < N; c0 += 64) {
                     uint32_t r[32];
+                    const bool stamp = et == 0 && acc_i == 0;
                     tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
                     tmem_ld_wait();
+                    if (stamp) GR_TRACE(kGtSliceBase + 4 * (c0 >> 5));
+                    __nv_bfloat16 hb[32];
                     if (sg.kind == 0) {
+                        // the slice's gates and bits into registers first: loads from
+                        // shared memory interleaved with the staging stores would each
+                        // wait for the store before them (the compiler cannot tell the
+                        // two shared arrays apart), serialising the 32 tokens
                         const uint32_t bits = sh.s_bits[c0 >> 5];
+                        float gv[32];
+#pragma unroll
+                        for (int u4 = 0; u4 < 8; ++u4) {
+                            const float4 g4 = reinterpret_cast<const float4*>(sh.s_gv + c0)[u4];
+                            gv[4 * u4] = g4.x;
+                            gv[4 * u4 + 1] = g4.y;
+                            gv[4 * u4 + 2] = g4.z;
+                            gv[4 * u4 + 3] = g4.w;
+                        }
 #pragma unroll
                         for (int u = 0; u < 32; ++u) {
-                            const float h = ((bits >> u) & 1u) ? sh.s_gv[c0 + u] * gr_swish(__uint_as_float(r[u])) : 0.f;
-                            stg[u * 128 + row] = __float2bfloat16_rn(h);
+                            const float h = ((bits >> u) & 1u) ? gv[u] * gr_swish(__uint_as_float(r[u])) : 0.f;
+                            hb[u] = __float2bfloat16_rn(h);
                         }
                     } else {
 #pragma unroll
-                        for (int u = 0; u < 32; ++u) stg[u * 128 + row] = __float2bfloat16_rn(__uint_as_float(r[u]));
+                        for (int u = 0; u < 32; ++u) hb[u] = __float2bfloat16_rn(__uint_as_float(r[u]));
                     }
-                    named_bar_sync(1, 128);
+                    // the group's previous slice has been copied out (barrier below)
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) stg[u * 128 + row] = hb[u];
+                    if (stamp) GR_TRACE(kGtSliceBase + 4 * (c0 >> 5) + 1);
+                    named_bar_sync(2 + eg, 128);
+                    if (stamp) GR_TRACE(kGtSliceBase + 4 * (c0 >> 5) + 2);
                     if (et == 0 && acc_i == 0 && c0 == 0) GR_TRACE(kGtFirstSlice);
-                    // 32 tokens x 16 pieces of 16 bytes; (the other staging slice is
-                    // being filled meanwhile, so one barrier per slice suffices)
+                    // 32 tokens x 16 pieces of 16 bytes
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const int c = et + 128 * k;
+                        const int c = gt + 128 * k;
                         const int tok = c >> 4, piece = c & 15;
                         if (c0 + tok < ntok)
                             *reinterpret_cast<uint4*>(dst + (size_t)(c0 + tok) * ld + piece * 8) =
                                 reinterpret_cast<const uint4*>(stg + tok * 128)[piece];
                     }
+                    named_bar_sync(2 + eg, 128);   // the staging slice is free again
+                    if (stamp) GR_TRACE(kGtSliceBase + 4 * (c0 >> 5) + 3);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.acc_empty[ab]);
                 if (et == 0 && acc_i == 0) GR_TRACE(kGtADrained);
                 ++acc_i;
-                if (sg.kind == 0) named_bar_sync(1, 128);   // the staged gates are free again
+                if (sg.kind == 0) named_bar_sync(1, kGrEpi);   // the staged gates are free again
             } else {
                 // publish this block's partial tile and count it in; the slice is
-                // finished in the second pass.  Layout: float4 (token quad k, row)
-                // at k * 128 + row.
-                // (only expert-out units are ever split)
+                // finished after the last accumulator.  Layout: float4 (token quad
+                // k, row) at k * 128 + row.  (Only expert-out units are ever split.)
                 float* part = a.partB;
                 const int myslot = bLo >= sg.first ? 0 : 1;
                 float4* dst = reinterpret_cast<float4*>(part + (size_t)(cta * 2 + myslot) * (N * 128)) + row;
 #pragma unroll 1
-                for (int c0 = 0; c0 < N; c0 += 32) {
+                for (int c0 = 32 * eg; c0 < N; c0 += 64) {
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(tbase + (uint32_t)c0, r);
                     tmem_ld_wait();
@@ -730,11 +786,8 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.acc_empty[ab]);
                 ++acc_i;
-                if (npend < 2) {
-                    pend_sg[npend] = sg;
-                    pend_cb[npend] = cb;
-                    ++npend;
-                }
+                if (npend == 0) { pend_sg[0] = sg; pend_cb[0] = cb; ++npend; }
+                else if (npend == 1) { pend_sg[1] = sg; pend_cb[1] = cb; ++npend; }
             }
         }
         if (!failed && cur_kind == 0 && uHi > uLo) announce_a();   // expert-in work only
@@ -770,12 +823,18 @@ static cudaError_t launch_group_n(const GrArgs& a, const CUtensorMap* maps, int 
     cfg.blockDim = dim3(kGrThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    // One block per SM, all resident at once (blocks wait on one another's
+    // results, with bounded waits), and a programmatic dependent of the
+    // group-plan kernel: its blocks are scheduled while that kernel runs and
+    // start their set-up early.
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, union_expert_group<N>, maps[0], maps[1], maps[2], maps[3], a);
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, union_expert_group<N>, maps[0], maps[1], maps[2], maps[3], maps[4], a);
 }
 
 cudaError_t launch_forward_group(const GrArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s) {

@@ -71,7 +71,8 @@ struct GrArgs {
     unsigned long long* trace;   // optional [grid][64] globaltimer stamps (nullptr: off)
 };
 // maps: x [T, d_h] (box {64, N}), W_in [E*d_e, d_h] and W_out [E*d_h, d_e] (box
-// {64, 128}), h' [P*N, d_e] (box {64, N}); 2-D, bf16, 128-byte swizzle
+// {64, 128}), h' [P*N, d_e] (box {64, N}): 2-D, bf16, 128-byte swizzle; the
+// expert-out partial tiles as fp32 lines of 512 floats (box {128, N/4}, no swizzle)
 cudaError_t launch_forward_group(const GrArgs& a, const CUtensorMap* maps, int grid, cudaStream_t s);
 
 // Arguments of the single-chunk forward (see forward_decode.cu): expert-in

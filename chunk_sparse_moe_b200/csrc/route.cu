@@ -67,19 +67,19 @@ constexpr size_t route_smem_bytes() {
            (BF16 ? sizeof(__nv_bfloat16) * (size_t)(kRtTok + 64 * EV) * kRtRaw : 0);
 }
 
-// The cluster's KS partial logit tiles [kRtTok][EP] (one per block, in shared
+// The cluster's KS partial logit tiles [TOK][EP] (one per block, in shared
 // memory, complete: the caller has passed a cluster barrier) become gates: block
-// r takes tokens r*32/KS .. (r+1)*32/KS - 1, one warp per token; logit = sum over
+// r takes tokens r*TOK/KS .. (r+1)*TOK/KS - 1, one warp per token; logit = sum over
 // ranks 0..KS-1 of their partials (+ b_r), then ReLU, the mean of squares over E
 // and the scale.
-template <int EP>
+template <int EP, int TOK = kRtTok>
 __device__ __forceinline__ void route_finish(const float* part, int KS, int r, int t0, int Ttok, int E,
                                              const float* __restrict__ b_r, const float* __restrict__ gamma,
                                              float eps, float* __restrict__ gates) {
     constexpr int NJ = EP / 32;   // experts per lane
     const int tid = threadIdx.x;
 
-    const int tpb = kRtTok / KS;
+    const int tpb = TOK / KS;
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t part_u32 = smem_u32(part);
     for (int tt = warp; tt < tpb; tt += (int)(blockDim.x / 32)) {
@@ -235,9 +235,12 @@ constexpr int kRqThreads = 128;
 constexpr int kRqKg = 256;                   // k per group
 constexpr uint64_t kRqWaitNs = 2000000000ull;
 
-template <int ET>
+// TOK tokens per cluster: 32 for short inputs (a decode step), 128 for long ones,
+// where the W_r tiles are then reused over four times as many tokens and the grid
+// has a quarter of the clusters (one wave at 4096 tokens).
+template <int ET, int TOK>
 constexpr size_t route_tc_smem_bytes() {
-    return 1024 + (size_t)ET * 65536 + 16384 + sizeof(float) * kRtTok * 128 * ET;
+    return 1024 + (size_t)ET * 65536 + (size_t)TOK * 512 + sizeof(float) * TOK * 128 * ET;
 }
 
 __device__ __forceinline__ bool rq_wait(uint64_t* bar, uint32_t parity) {
@@ -248,23 +251,24 @@ __device__ __forceinline__ bool rq_wait(uint64_t* bar, uint32_t parity) {
     return true;
 }
 
-template <int ET>
+template <int ET, int TOK>
 __global__ void __launch_bounds__(kRqThreads, 1) route_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
     const float* __restrict__ b_r, const float* __restrict__ gamma, float eps, int Ttok, int E, int KS,
     int slice, float* __restrict__ gates) {
     constexpr int EP = 128 * ET;
-    constexpr uint32_t kCols = 32 * ET;   // one 32-column accumulator per expert tile (a power of 2)
+    constexpr uint32_t kCols = TOK * ET;  // one TOK-column accumulator per expert tile (a power of 2)
+    constexpr int kXBytes = TOK * 512;    // x box: 4 k-blocks of TOK rows x 128 B
     extern __shared__ uint8_t rq_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rq_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* wsm = sm;                                   // [ET][4 k-blocks][128 rows x 128 B]
-    uint8_t* xsm = sm + ET * 65536;                      // [4 k-blocks][32 rows x 128 B]
-    float* part = reinterpret_cast<float*>(xsm + 16384);  // [kRtTok][EP]
+    uint8_t* xsm = sm + ET * 65536;                      // [4 k-blocks][TOK rows x 128 B]
+    float* part = reinterpret_cast<float*>(xsm + kXBytes);  // [TOK][EP]
     __shared__ __align__(8) uint64_t full, mma_bar;
     __shared__ uint32_t tmem_base;
     __shared__ int ok_s;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * kRtTok;
+    const int t0 = blockIdx.x * TOK;
     const int r = (int)cluster_ctarank();
     if (threadIdx.x == 0) {
         mbar_init(&full, 1);
@@ -284,14 +288,14 @@ __global__ void __launch_bounds__(kRqThreads, 1) route_tc_kernel(
     griddep_launch_dependents();
     const uint32_t tmem = tmem_base;
     if (threadIdx.x == 0) {
-        const uint32_t idesc = idesc_bf16_f32(128, kRtTok);
+        const uint32_t idesc = idesc_bf16_f32(128, TOK);
         const uint64_t pol = policy_evict_last();
         const uint64_t dw = sw128_kmajor_desc(smem_u32(wsm)), dx = sw128_kmajor_desc(smem_u32(xsm));
         bool ok = true;
         const int ng = slice / kRqKg;
         for (int g = 0; g < ng && ok; ++g) {
             const int kb0 = (r * slice + g * kRqKg) / 64;
-            mbar_arrive_expect_tx(&full, (uint32_t)(ET * 65536 + 16384));
+            mbar_arrive_expect_tx(&full, (uint32_t)(ET * 65536 + kXBytes));
 #pragma unroll
             for (int et = 0; et < ET; ++et) tma_load_3d(wsm + et * 65536, &tm_w, &full, 0, et * 128, kb0, pol);
             tma_load_3d(xsm, &tm_x, &full, 0, t0, kb0, pol);
@@ -304,9 +308,9 @@ __global__ void __launch_bounds__(kRqThreads, 1) route_tc_kernel(
                 for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(tmem + (uint32_t)(32 * et),
+                        umma_bf16(tmem + (uint32_t)(TOK * et),
                                   dw + (uint64_t)((et * 65536 + kb * 16384 + kk * 32) >> 4),
-                                  dx + (uint64_t)((kb * 4096 + kk * 32) >> 4), idesc,
+                                  dx + (uint64_t)((kb * TOK * 128 + kk * 32) >> 4), idesc,
                                   (g > 0 || kb > 0 || kk > 0) ? 1u : 0u);
             umma_commit(&mma_bar);
             // the buffers are reloaded (next group) or the accumulators read only
@@ -326,17 +330,20 @@ __global__ void __launch_bounds__(kRqThreads, 1) route_tc_kernel(
     const bool ok = ok_s != 0;
     // accumulator row = TMEM lane = expert (warp w holds experts 32w .. 32w+31 of each tile)
 #pragma unroll
-    for (int et = 0; et < ET; ++et) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * et), v);
-        tmem_ld_wait();
-        const int e = 128 * et + 32 * warp + lane;
+    for (int et = 0; et < ET; ++et)
+#pragma unroll 1
+        for (int c0 = 0; c0 < TOK; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(TOK * et + c0), v);
+            tmem_ld_wait();
+            const int e = 128 * et + 32 * warp + lane;
 #pragma unroll
-        for (int t = 0; t < kRtTok; ++t) part[t * EP + e] = ok ? __uint_as_float(v[t]) : __int_as_float(0x7fc00000);
-    }
+            for (int t = 0; t < 32; ++t)
+                part[(c0 + t) * EP + e] = ok ? __uint_as_float(v[t]) : __int_as_float(0x7fc00000);
+        }
     tc_fence_before();
     cluster_barrier_sync();   // every block's partials are written
-    route_finish<EP>(part, KS, r, t0, Ttok, E, b_r, gamma, eps, gates);
+    route_finish<EP, TOK>(part, KS, r, t0, Ttok, E, b_r, gamma, eps, gates);
     cluster_barrier_sync();   // no block leaves while a peer may still read its partials
     if (warp == 0) {
         tc_fence_after();
@@ -344,20 +351,20 @@ __global__ void __launch_bounds__(kRqThreads, 1) route_tc_kernel(
     }
 }
 
-template <int ET>
+template <int ET, int TOK>
 static cudaError_t launch_route_tc(const __nv_bfloat16* x, const __nv_bfloat16* W_r, const float* b_r,
                                    const float* gamma, float eps, int Ttok, int d_h, int E, int KS, float* gates,
                                    cudaStream_t s) {
     CUtensorMap mx, mw;
-    if (!make_map_kblocks(&mx, x, (uint64_t)d_h, (uint64_t)Ttok, kRtTok, 4) ||
+    if (!make_map_kblocks(&mx, x, (uint64_t)d_h, (uint64_t)Ttok, TOK, 4) ||
         !make_map_kblocks(&mw, W_r, (uint64_t)d_h, (uint64_t)E, 128, 4))
         return cudaErrorInvalidValue;
-    const size_t smem = route_tc_smem_bytes<ET>();
+    const size_t smem = route_tc_smem_bytes<ET, TOK>();
     cudaError_t err =
-        cudaFuncSetAttribute(route_tc_kernel<ET>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(route_tc_kernel<ET, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((Ttok + kRtTok - 1) / kRtTok, KS, 1);
+    cfg.gridDim = dim3((Ttok + TOK - 1) / TOK, KS, 1);
     cfg.blockDim = dim3(kRqThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -368,7 +375,8 @@ static cudaError_t launch_route_tc(const __nv_bfloat16* x, const __nv_bfloat16* 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, route_tc_kernel<ET>, mx, mw, b_r, gamma, eps, Ttok, E, KS, d_h / KS, gates);
+    return cudaLaunchKernelEx(&cfg, route_tc_kernel<ET, TOK>, mx, mw, b_r, gamma, eps, Ttok, E, KS, d_h / KS,
+                              gates);
 }
 
 template <typename T, int EV>
@@ -411,13 +419,19 @@ cudaError_t launch_route(const void* x, const void* W_r, const float* b_r, const
                          cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     if (bf16 && d_h % kRqKg == 0 && E <= 256) {
-        // tensor cores: KS slices of whole 256-k groups
-        int KS = kRtMaxKS;
-        while (KS > 1 && d_h % (kRqKg * KS) != 0) KS /= 2;
+        // tensor cores: KS slices of whole 256-k groups; long inputs (E <= 128)
+        // take 128 tokens per cluster of at most 4 blocks
         const auto* xb = static_cast<const __nv_bfloat16*>(x);
         const auto* wb = static_cast<const __nv_bfloat16*>(W_r);
-        return E <= 128 ? launch_route_tc<1>(xb, wb, b_r, gamma, eps, T, d_h, E, KS, gates, s)
-                        : launch_route_tc<2>(xb, wb, b_r, gamma, eps, T, d_h, E, KS, gates, s);
+        if (T >= 1024 && E <= 128) {
+            int KS = 4;
+            while (KS > 1 && d_h % (kRqKg * KS) != 0) KS /= 2;
+            return launch_route_tc<1, 128>(xb, wb, b_r, gamma, eps, T, d_h, E, KS, gates, s);
+        }
+        int KS = kRtMaxKS;
+        while (KS > 1 && d_h % (kRqKg * KS) != 0) KS /= 2;
+        return E <= 128 ? launch_route_tc<1, kRtTok>(xb, wb, b_r, gamma, eps, T, d_h, E, KS, gates, s)
+                        : launch_route_tc<2, kRtTok>(xb, wb, b_r, gamma, eps, T, d_h, E, KS, gates, s);
     }
     if (bf16)
         return launch_route_t(static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(W_r), b_r,

@@ -185,39 +185,59 @@ cudaError_t launch_chunk_union_plan(const float* gates, int T, int E, int n, int
     return cudaGetLastError();
 }
 
-// Group tables of the multi-chunk forward (forward_group.cu).  Groups are NG
-// consecutive chunks; a group's expert set is the union of its chunks' unions,
-// ascending: e is in it when some chunk of the group has a nonzero token mask
-// for e.  One block of 1024 threads:
-//   1. the per-chunk tables, computed from the gates, or the caller's checked;
-//   2. gcounts[g] = size of group g's set (warp per group, ballot per 32 experts);
-//   3. goffsets = exclusive scan of gcounts;
-//   4. gpair[goffsets[g] + s] = (g << 8) | (s-th expert of the set), and the rows
-//      of y of a group with an empty set zeroed (no later kernel writes them).
+// Group tables of the multi-chunk forward (forward_group.cu), one launch.  Groups
+// are NG consecutive chunks; a group's expert set is the union of its chunks'
+// unions, ascending: e is in it when some chunk of the group has a nonzero
+// token mask for e.
+//   1. every warp takes one chunk: its tables from the gates (union_one_chunk),
+//      or the caller's tables checked against their token masks;
+//   2. the last block to finish (a counter in the control block, reset by that
+//      block for the next launch) builds the group tables: gcounts[g], their
+//      exclusive scan goffsets, gpair[goffsets[g] + s] = (g << 8) | (s-th expert
+//      of the set), and zeroes the rows of y of a group whose set is empty (no
+//      later kernel writes them).
+// Launched as a programmatic dependent of the previous kernel (the router, when
+// the gates come from it): it waits for that kernel before reading the gates,
+// and lets the group kernel, its own dependent, be scheduled at once.
 __device__ __forceinline__ bool group_has(const uint32_t* tmask, int E, int C, int NG, int g, int e) {
     bool any = false;
     if (e < E) {
         const int c1 = min(C, (g + 1) * NG);
-        for (int c = g * NG; c < c1; ++c) any = any || tmask[(size_t)c * E + e] != 0u;
+        for (int c = g * NG; c < c1; ++c) any = any || __ldcg(tmask + (size_t)c * E + e) != 0u;
     }
     return any;
 }
 
-__global__ void __launch_bounds__(1024) group_plan_kernel(
-    const float* __restrict__ gates, int T, int E, int n, int C, int32_t* counts, int32_t* idx,
-    uint32_t* tmask, int compute_union, Ctl* ctl, int NG, int NGr, int32_t* __restrict__ gcounts,
-    int32_t* __restrict__ goffsets, int32_t* __restrict__ gpair, __nv_bfloat16* __restrict__ y, int d_h) {
+constexpr int kGpThreads = 256;
+
+__global__ void __launch_bounds__(kGpThreads) group_union_plan_kernel(
+    const float* __restrict__ gates, int T, int E, int n, int C, int32_t* counts, int32_t* idx, uint32_t* tmask,
+    int compute_union, Ctl* ctl, int NG, int NGr, int32_t* __restrict__ gcounts, int32_t* __restrict__ goffsets,
+    int32_t* __restrict__ gpair, __nv_bfloat16* __restrict__ y, int d_h) {
+    __shared__ int s_last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
-    if (compute_union) {
-        for (int c = warp; c < C; c += nwarps) union_one_chunk(gates, T, E, n, c, lane, counts, idx, tmask);
-    } else {
-        for (int c = warp; c < C; c += nwarps) check_one_chunk(E, c, lane, counts, idx, tmask, ctl);
+    griddep_wait();
+    if (threadIdx.x == 0) griddep_launch_dependents();
+    const int c = blockIdx.x * nwarps + warp;
+    if (c < C) {
+        if (compute_union) union_one_chunk(gates, T, E, n, c, lane, counts, idx, tmask);
+        else check_one_chunk(E, c, lane, counts, idx, tmask, ctl);
     }
-    if (plan_refused(ctl)) return;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();   // this block's tables before its count
+        s_last = atomicAdd(&ctl->plan_done, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();       // every block's tables after the count that saw them all
+    if (threadIdx.x == 0) ctl->plan_done = 0u;
+    if (plan_refused(ctl)) return;   // refused tables or an earlier error: compute nothing
     for (int g = warp; g < NGr; g += nwarps) {
         int base = 0;
-        for (int g0 = 0; g0 < E; g0 += 32) base += __popc(__ballot_sync(0xffffffffu, group_has(tmask, E, C, NG, g, g0 + lane)));
+        for (int g0 = 0; g0 < E; g0 += 32)
+            base += __popc(__ballot_sync(0xffffffffu, group_has(tmask, E, C, NG, g, g0 + lane)));
         if (lane == 0) gcounts[g] = base;
     }
     __syncthreads();
@@ -247,9 +267,17 @@ cudaError_t launch_group_plan(const float* gates, int T, int E, int n, int32_t* 
                               int d_h, cudaStream_t s) {
     const int C = (T + n - 1) / n;
     if (C == 0) return cudaSuccess;
-    group_plan_kernel<<<1, 1024, 0, s>>>(gates, T, E, n, C, counts, idx, tmask, compute_union ? 1 : 0, ctl,
-                                         NG, NGr, gcounts, goffsets, gpair, y, d_h);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((C + kGpThreads / 32 - 1) / (kGpThreads / 32));
+    cfg.blockDim = dim3(kGpThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, group_union_plan_kernel, gates, T, E, n, C, counts, idx, tmask,
+                              compute_union ? 1 : 0, ctl, NG, NGr, gcounts, goffsets, gpair, y, d_h);
 }
 
 }  // namespace bffn

@@ -253,20 +253,22 @@ void blockffn_debug_skip_flag(int unit);
 /*
  * blockffn_debug_set_trace -- timeline tracing of later bf16 forward launches.
  * device_buffer (device memory, zeroed by the caller, blockffn_num_sms() * 64
- * uint64 entries) receives globaltimer stamps in nanoseconds, per thread block.
- * Multi-chunk launches use 32 entries per block: 0 start, 1 prologue done,
- * 2 first weight load issued, 3 last load issued, 4 first tile landed, 5 last
- * expert-in accumulator committed, 6 first accumulator drained, 7 last expert-in
- * unit finished, 8 first and 9 last activation flag seen, 10 last accumulator
- * committed, 11 last unit finished, 12 teardown, 13 end; for the block's first
- * expert-in (A) and expert-out (B) unit: 14/21 partial written, 15/22 arrival
- * counted, 16/23 partials summed, 17 activations published; 18 gates loaded,
- * 19 control word loaded, 20 TMEM allocated, 24 first activation tile copied,
- * 25 first expert-out MMA issued.
- * Single-chunk launches use 64 entries per block: 0 start, 1 prologue done,
+ * uint64 entries) receives globaltimer stamps in nanoseconds, 64 entries per
+ * thread block.
+ * Multi-chunk (group) launches: 0 start, 1 prologue done, 2 first weight load
+ * issued, 3 last expert-in weight load issued, 4 last expert-in accumulator
+ * committed, 5 expert-in results announced, 6 first expert-out activation tile
+ * ready, 7 last expert-out accumulator committed, 8 epilogue done, 9 end,
+ * 10 first accumulator drained, 12 last load issued, 13 first expert-in
+ * accumulator written out, 14 expert-in announcement begun, 15 first 32-token
+ * slice staged; for the first unit's slices s = 0..7, 16 + 4s + {0: TMEM read,
+ * 1: staged, 2: barrier passed, 3: stores issued}; 48 expert-out partials
+ * written, 49 announced, and for pending split unit k = 0, 1: 50 + 3k
+ * contributors counted, 51 + 3k partials summed, 52 + 3k rows of y stored.
+ * Single-chunk launches: 0 start, 1 prologue done,
  * 2 first weight load issued, 3 last load issued, 4 first expert-in tile landed,
  * 5 last expert-in accumulator committed, 7 expert-in units finished, 8 first and
- * 9 last time every h' slot was seen ready, 10 last expert-out accumulator
+ * 9 last expert slot seen ready, 10 last expert-out accumulator
  * committed, 11 last epilogue step, 13 end; for the block's first expert-in unit:
  * 14 accumulator read, 15 partial sent to the peer, 16 peer's partial received,
  * 17 peer's partial read, 18 h' published; 21 first expert-out quadrant sent,

@@ -94,6 +94,8 @@ def test_route_seq4096_bf16(bffn):
     (7, 4096, 256, None),    # fewer tokens than a tile, two 256-wide k-groups per slice
     (70, 2304, 64, -0.5),    # d_h 9 x 256: one slice of nine k-groups
     (33, 320, 48, None),     # d_h not a multiple of 256: the CUDA-core router
+    (1100, 1024, 48, -0.8),  # long input: 128 tokens per cluster of 4, ragged last tile
+    (2000, 512, 128, None),  # long input, d_h in 2 slices, all 128 expert rows
 ])
 def test_route_bf16_shapes(bffn, T, d_h, E, bias):
     w = wl.make_routed("route_shape", T, 32, d_h, E, 1, "bf16", seed=T + E, bias_shift=bias)
