@@ -12,6 +12,7 @@ passages they follow:
 * ``route``               -- g = RMSNorm(ReLU(W_r x + b_r)) over the expert axis
 * ``chunk_union``         -- per-chunk union of active experts, token bitmasks
 * ``forward_dense``       -- y = sum over ALL experts of gate * expert(x)
+                             (expert biases optional)
 * ``forward_chunk_union`` -- union experts over whole chunks, masked after compute
 * ``sparsity``            -- token-level and L-token chunk-level sparsity
 * ``residual_layernorm``  -- LayerNorm(y + x) over the hidden dimension
@@ -62,9 +63,9 @@ def _load():
                                      ctypes.c_int, ctypes.c_int, _D, _D]
         lib.oracle_chunk_union.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            _I32, _I32, _U32]
-        lib.oracle_forward_dense.argtypes = [_D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
+        lib.oracle_forward_dense.argtypes = [_D, _D, _D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_int, _D]
-        lib.oracle_forward_chunk_union.argtypes = [_D, _D, _D, _D, ctypes.c_int,
+        lib.oracle_forward_chunk_union.argtypes = [_D, _D, _D, _D, _D, _D, ctypes.c_int,
                                                    ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, _D]
         lib.oracle_sparsity.argtypes = [_D, ctypes.c_int, ctypes.c_int, ctypes.c_int, _D]
@@ -117,29 +118,44 @@ def chunk_union(gates, n: int):
     return counts, idx, tmask
 
 
-def forward_dense(x, gates, W_in, W_out) -> np.ndarray:
-    """y = sum over all experts of gate * W_out_e Swish(W_in_e x), fp64."""
+def _biases(b_in, b_out, E, d_e, d_h):
+    bi = None if b_in is None else _f64(b_in)
+    bo = None if b_out is None else _f64(b_out)
+    assert bi is None or bi.shape == (E, d_e)
+    assert bo is None or bo.shape == (E, d_h)
+    return bi, bo
+
+
+def forward_dense(x, gates, W_in, W_out, b_in=None, b_out=None) -> np.ndarray:
+    """y = sum over all experts of gate * (W_out_e Swish(W_in_e x + b_in_e) + b_out_e),
+    fp64; b_in [E, d_e] and b_out [E, d_h] are optional (absent = no bias)."""
     lib = _load()
     x, g, W_in, W_out = _f64(x), _f64(gates), _f64(W_in), _f64(W_out)
     T, d_h = x.shape
     E, d_e, _ = W_in.shape
     assert W_in.shape == (E, d_e, d_h) and W_out.shape == (E, d_h, d_e) and g.shape == (T, E)
+    bi, bo = _biases(b_in, b_out, E, d_e, d_h)
     y = np.empty((T, d_h), np.float64)
     lib.oracle_forward_dense(_p(x, _D), _p(g, _D), _p(W_in, _D), _p(W_out, _D),
+                             None if bi is None else _p(bi, _D), None if bo is None else _p(bo, _D),
                              T, d_h, E, d_e, _p(y, _D))
     return y
 
 
-def forward_chunk_union(x, gates, W_in, W_out, n: int) -> np.ndarray:
-    """Union experts over whole n-token chunks, masked after computing, fp64."""
+def forward_chunk_union(x, gates, W_in, W_out, n: int, b_in=None, b_out=None) -> np.ndarray:
+    """Union experts over whole n-token chunks, masked after computing, fp64
+    (expert biases optional, as in ``forward_dense``)."""
     lib = _load()
     x, g, W_in, W_out = _f64(x), _f64(gates), _f64(W_in), _f64(W_out)
     T, d_h = x.shape
     E, d_e, _ = W_in.shape
     assert W_in.shape == (E, d_e, d_h) and W_out.shape == (E, d_h, d_e) and g.shape == (T, E)
     assert 1 <= n <= 32
+    bi, bo = _biases(b_in, b_out, E, d_e, d_h)
     y = np.empty((T, d_h), np.float64)
     lib.oracle_forward_chunk_union(_p(x, _D), _p(g, _D), _p(W_in, _D), _p(W_out, _D),
+                                   None if bi is None else _p(bi, _D),
+                                   None if bo is None else _p(bo, _D),
                                    T, d_h, E, d_e, n, _p(y, _D))
     return y
 

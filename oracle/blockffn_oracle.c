@@ -23,8 +23,8 @@
  *   W_r    [E, d_h]          router weight;  b_r [E] optional router bias
  *   gamma  [E]               RMSNorm scale
  *   gates  [T, E]
- *   W_in   [E, d_e, d_h]     expert fc1 weights
- *   W_out  [E, d_h, d_e]     expert fc2 weights
+ *   W_in   [E, d_e, d_h]     expert fc1 weights;  b_in  [E, d_e] optional fc1 biases
+ *   W_out  [E, d_h, d_e]     expert fc2 weights;  b_out [E, d_h] optional fc2 biases
  *   y      [T, d_h]
  */
 #include <math.h>
@@ -123,12 +123,16 @@ static double silu(double z) { return z / (1.0 + exp(-z)); }
 
 /*
  * One expert on one token.  [SKILL] "Router Architecture Setup" (expert module:
- * fc1 -> SiLU -> dropout -> fc2) and "Architecture Overview" (non-gated MLP with
- * Swish, d_e << d_h).  Inference: dropout is the identity.  Biases are not part
- * of the layer here (the expert is W_out_e * Swish(W_in_e x)).
- *   h[j] = silu( sum_k W_in[e,j,k] x[k] ),  o[i] = sum_j W_out[e,i,j] h[j]
+ * fc1 -> SiLU -> dropout -> fc2, both nn.Linear) and "Architecture Overview"
+ * (non-gated MLP with Swish, d_e << d_h).  Inference: dropout is the identity.
+ * nn.Linear carries a bias by default; the biases are optional here (NULL = the
+ * expert is W_out_e Swish(W_in_e x), the form the layer's sparse computation is
+ * stated in):
+ *   h[j] = silu( sum_k W_in[e,j,k] x[k] + b_in[e,j] ),
+ *   o[i] = sum_j W_out[e,i,j] h[j] + b_out[e,i]
  */
 static void expert_apply(const double* xt, const double* W_in, const double* W_out,
+                         const double* b_in, const double* b_out,
                          int d_h, int d_e, int e, double* h, double* o)
 {
     const double* Wi = W_in + (size_t)e * d_e * d_h;
@@ -136,11 +140,13 @@ static void expert_apply(const double* xt, const double* W_in, const double* W_o
     for (int j = 0; j < d_e; ++j) {
         double s = 0.0;
         for (int k = 0; k < d_h; ++k) s += Wi[(size_t)j * d_h + k] * xt[k];
+        if (b_in) s += b_in[(size_t)e * d_e + j];
         h[j] = silu(s);
     }
     for (int i = 0; i < d_h; ++i) {
         double s = 0.0;
         for (int j = 0; j < d_e; ++j) s += Wo[(size_t)i * d_e + j] * h[j];
+        if (b_out) s += b_out[(size_t)e * d_h + i];
         o[i] = s;
     }
 }
@@ -151,12 +157,14 @@ static void expert_apply(const double* xt, const double* W_in, const double* W_o
  * token, each output is multiplied by that token's gate, and the products are
  * summed over the experts.  The gate is g = RMSNorm(ReLU(W_r x)) ([ABS]), not the
  * sigmoid training probabilities; the LayerNorm + residual that follows the sum
- * on that page is outside the FFN output y.
+ * on that page is outside the FFN output y.  The gate multiplies the whole
+ * expert output, its fc2 bias included.
  *
- *   y[t,:] = sum_{e=0}^{E-1} gates[t,e] * W_out_e Swish(W_in_e x_t)
+ *   y[t,:] = sum_{e=0}^{E-1} gates[t,e] * ( W_out_e Swish(W_in_e x_t + b_in_e) + b_out_e )
  */
 void oracle_forward_dense(const double* x, const double* gates, const double* W_in,
-                          const double* W_out, int T, int d_h, int E, int d_e, double* y)
+                          const double* W_out, const double* b_in, const double* b_out,
+                          int T, int d_h, int E, int d_e, double* y)
 {
     int t;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -167,7 +175,7 @@ void oracle_forward_dense(const double* x, const double* gates, const double* W_
         for (int i = 0; i < d_h; ++i) yt[i] = 0.0;
         for (int e = 0; e < E; ++e) {
             double g = gates[(size_t)t * E + e];
-            expert_apply(x + (size_t)t * d_h, W_in, W_out, d_h, d_e, e, h, o);
+            expert_apply(x + (size_t)t * d_h, W_in, W_out, b_in, b_out, d_h, d_e, e, h, o);
             for (int i = 0; i < d_h; ++i) yt[i] += g * o[i];
         }
         free(h);
@@ -185,12 +193,13 @@ void oracle_forward_dense(const double* x, const double* gates, const double* W_
  *
  *   y[t,:] = sum_{e in U_c, ascending} ( bit_t(tmask[c,e]) ? gates[t,e] * o_e(x_t) : 0 )
  *
+ * with o_e the expert's output as above (its biases included when given).
  * Masked terms are selected to exactly zero.  Same summation order as the dense
  * definition restricted to the active experts.
  */
 void oracle_forward_chunk_union(const double* x, const double* gates, const double* W_in,
-                                const double* W_out, int T, int d_h, int E, int d_e, int n,
-                                double* y)
+                                const double* W_out, const double* b_in, const double* b_out,
+                                int T, int d_h, int E, int d_e, int n, double* y)
 {
     int C = (T + n - 1) / n;
     int32_t* counts = (int32_t*)malloc(sizeof(int32_t) * (size_t)C);
@@ -207,7 +216,7 @@ void oracle_forward_chunk_union(const double* x, const double* gates, const doub
         for (int s = 0; s < counts[c]; ++s) {
             int e = idx[(size_t)c * E + s];
             uint32_t bits = tmask[(size_t)c * E + e];
-            expert_apply(x + (size_t)t * d_h, W_in, W_out, d_h, d_e, e, h, o);
+            expert_apply(x + (size_t)t * d_h, W_in, W_out, b_in, b_out, d_h, d_e, e, h, o);
             int keep = (int)((bits >> j) & 1u);
             double g = gates[(size_t)t * E + e];
             for (int i = 0; i < d_h; ++i)

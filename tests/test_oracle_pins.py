@@ -13,12 +13,15 @@ from a fact the pages or mathematics fix:
 * the router equals torch's own ``rms_norm`` of ``relu(W_r x + b)``;
 * hand-derived worked examples (tests/golden/hand_examples.json);
 * the residual LayerNorm equals torch's ``layer_norm`` of y + x, and its closed
-  forms (constant row -> shift, unit moments, scale invariance).
+  forms (constant row -> shift, unit moments, scale invariance);
+* with expert biases: the concatenated-expert MLP with biases (numpy), the
+  x = 0 closed form, and the pages' expert module built from torch nn.Linear.
 
 ``test_pins_catch_planted_mistakes`` compiles mutated copies of the oracle
 (a dropped expert, a sign flip in Swish, a transposed weight index, the wrong
 token's gate, a wrong RMS mean, a shifted token bit, a scrambled union list, a
-LayerNorm without the residual, a sample variance)
+LayerNorm without the residual, a sample variance, an fc1 bias after the
+activation or from the wrong expert, a dropped or ungated fc2 bias)
 and checks that at least one pin fails for each.
 """
 from __future__ import annotations
@@ -118,6 +121,80 @@ def pin_union_then_mask(orc) -> float:
         # non-zero terms in the same order, so they agree bit for bit
         exact = 0.0 if np.array_equal(yd, yu) else 1.0
         worst = max(worst, exact, _rel(yd, ys))
+    return worst
+
+
+def _rand_biases(seed, E, d_e, d_h, scale=0.5):
+    rng = np.random.default_rng(500 + seed)
+    return scale * rng.standard_normal((E, d_e)), scale * rng.standard_normal((E, d_h))
+
+
+def pin_bias_all_on_mlp(orc) -> float:
+    """Expert biases, gates all non-zero: the layer is one MLP over the
+    concatenated experts, y = W_out_cat (g_rep * Swish(W_in_cat x + b_in_cat))
+    + g B_out (numpy matmuls), in the dense definition and the union schedule."""
+    worst = 0.0
+    for seed in range(3):
+        x, W_in, W_out = _rand_problem(seed, d_e=5)
+        T, E, d_e, d_h = x.shape[0], W_in.shape[0], W_in.shape[1], W_in.shape[2]
+        b_in, b_out = _rand_biases(seed, E, d_e, d_h)
+        rng = np.random.default_rng(300 + seed)
+        gates = rng.uniform(0.1, 2.0, (T, E))
+        W_in_cat = W_in.reshape(E * d_e, d_h)
+        W_out_cat = np.concatenate(list(W_out), axis=1)
+        hidden = _silu(x @ W_in_cat.T + b_in.reshape(-1)) * np.repeat(gates, d_e, axis=1)
+        y_ref = hidden @ W_out_cat.T + gates @ b_out
+        worst = max(worst, _rel(orc.forward_dense(x, gates, W_in, W_out, b_in, b_out), y_ref))
+        worst = max(worst, _rel(orc.forward_chunk_union(x, gates, W_in, W_out, 4, b_in, b_out), y_ref))
+    return worst
+
+
+def pin_bias_zero_input(orc) -> float:
+    """x = 0: every expert outputs W_out_e Swish(b_in_e) + b_out_e, so
+    y_t = sum_e g_te (W_out_e Swish(b_in_e) + b_out_e) (closed form)."""
+    x, W_in, W_out = _rand_problem(21, d_e=3)
+    x = np.zeros_like(x)
+    T, E, d_e, d_h = x.shape[0], W_in.shape[0], W_in.shape[1], W_in.shape[2]
+    b_in, b_out = _rand_biases(21, E, d_e, d_h, scale=1.0)
+    rng = np.random.default_rng(22)
+    gates = np.where(rng.random((T, E)) < 0.5, rng.uniform(-1.0, 2.0, (T, E)), 0.0)
+    per_expert = np.stack([W_out[e] @ _silu(b_in[e]) + b_out[e] for e in range(E)])   # [E, d_h]
+    y_ref = gates @ per_expert
+    worst = _rel(orc.forward_dense(x, gates, W_in, W_out, b_in, b_out), y_ref)
+    return max(worst, _rel(orc.forward_chunk_union(x, gates, W_in, W_out, 2, b_in, b_out), y_ref))
+
+
+def pin_bias_torch_modules(orc) -> float:
+    """The expert as the pages build it -- fc1 = nn.Linear(d_h, d_e), SiLU,
+    fc2 = nn.Linear(d_e, d_h), biases on -- in torch fp64, gated and summed over
+    the experts with sparse gates; against both oracle schedules.  Zero biases
+    give the bias-free forward exactly."""
+    import torch
+    worst = 0.0
+    for seed, n in [(31, 3), (32, 5)]:
+        x, W_in, W_out = _rand_problem(seed, T=11, d_h=16, E=4, d_e=6)
+        T, E, d_e, d_h = x.shape[0], W_in.shape[0], W_in.shape[1], W_in.shape[2]
+        b_in, b_out = _rand_biases(seed, E, d_e, d_h)
+        rng = np.random.default_rng(seed)
+        gates = np.where(rng.random((T, E)) < 0.4, rng.uniform(0.2, 1.5, (T, E)), 0.0)
+        xt = torch.from_numpy(x)
+        y_ref = torch.zeros(T, d_h, dtype=torch.float64)
+        for e in range(E):
+            fc1 = torch.nn.Linear(d_h, d_e).double()
+            fc2 = torch.nn.Linear(d_e, d_h).double()
+            with torch.no_grad():
+                fc1.weight.copy_(torch.from_numpy(W_in[e]))
+                fc1.bias.copy_(torch.from_numpy(b_in[e]))
+                fc2.weight.copy_(torch.from_numpy(W_out[e]))
+                fc2.bias.copy_(torch.from_numpy(b_out[e]))
+                y_ref += torch.from_numpy(gates[:, e:e + 1]) * fc2(torch.nn.functional.silu(fc1(xt)))
+        y_ref = y_ref.numpy()
+        worst = max(worst, _rel(orc.forward_dense(x, gates, W_in, W_out, b_in, b_out), y_ref))
+        worst = max(worst, _rel(orc.forward_chunk_union(x, gates, W_in, W_out, n, b_in, b_out), y_ref))
+        z_in, z_out = np.zeros_like(b_in), np.zeros_like(b_out)
+        same = np.array_equal(orc.forward_chunk_union(x, gates, W_in, W_out, n, z_in, z_out),
+                              orc.forward_chunk_union(x, gates, W_in, W_out, n))
+        worst = max(worst, 0.0 if same else 1.0)
     return worst
 
 
@@ -319,6 +396,9 @@ PINS = {
     "sparsity": (pin_sparsity, 0.0),
     "residual_layernorm_torch": (pin_residual_layernorm_torch, 1e-13),
     "residual_layernorm_closed_forms": (pin_residual_layernorm_closed_forms, 1e-12),
+    "bias_all_on_mlp": (pin_bias_all_on_mlp, 1e-12),
+    "bias_zero_input": (pin_bias_zero_input, 1e-12),
+    "bias_torch_modules": (pin_bias_torch_modules, 1e-12),
 }
 
 
@@ -369,6 +449,16 @@ MUTANTS = {
                        "for (int k = 0; k < d_h; ++k) mu += yr[k];"),
     # the sample (n - 1) variance instead of nn.LayerNorm's population variance
     "ln_sample_variance": ("var /= (double)d_h;", "var /= (double)(d_h - 1);"),
+    # the fc1 bias added after the activation instead of before it
+    "bias_in_after_swish": ("if (b_in) s += b_in[(size_t)e * d_e + j];\n        h[j] = silu(s);",
+                            "h[j] = silu(s);\n        if (b_in) h[j] += b_in[(size_t)e * d_e + j];"),
+    # every expert reads expert 0's fc1 bias
+    "bias_in_wrong_expert": ("if (b_in) s += b_in[(size_t)e * d_e + j];", "if (b_in) s += b_in[j];"),
+    # the fc2 bias dropped
+    "bias_out_dropped": ("if (b_out) s += b_out[(size_t)e * d_h + i];", "if (b_out) s += 0.0;"),
+    # the fc2 bias added once per token outside the gate (ungated), not per expert
+    "bias_out_ungated": ("for (int i = 0; i < d_h; ++i) yt[i] += g * o[i];",
+                         "for (int i = 0; i < d_h; ++i) yt[i] += g * o[i] + (b_out ? b_out[(size_t)e * d_h + i] * (1.0 - g) : 0.0);"),
 }
 
 
