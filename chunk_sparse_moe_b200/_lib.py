@@ -23,6 +23,14 @@ c_void_p, c_int, c_float, c_size_t = ctypes.c_void_p, ctypes.c_int, ctypes.c_flo
 c_uint64 = ctypes.c_uint64
 c_int32_p = ctypes.POINTER(ctypes.c_int32)
 
+
+
+class LayerOpts(ctypes.Structure):
+    """blockffn_layer_opts: optional expert biases and closing LayerNorm."""
+    _fields_ = [("b_in", c_void_p), ("b_out", c_void_p), ("ln_weight", c_void_p),
+                ("ln_bias", c_void_p), ("ln_eps", c_float)]
+
+
 # name -> (restype, argtypes); every symbol include/blockffn.h declares
 SIGNATURES = {
     "blockffn_status_string": (ctypes.c_char_p, [c_int]),
@@ -40,7 +48,7 @@ SIGNATURES = {
     "blockffn_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float,
                                  c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
-                                 c_void_p, c_void_p, c_size_t, c_void_p]),
+                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "blockffn_get_device_status": (c_int, [c_void_p, c_void_p, c_int32_p]),
     "blockffn_forward_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                          c_int, c_int, c_int, c_void_p, c_void_p]),
@@ -58,3 +66,5 @@ for _name, (_res, _args) in SIGNATURES.items():
 # status codes and dtypes (include/blockffn.h)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(6)
 F32, BF16 = 0, 1
+# workspace-size flags
+WS_ROUTER, WS_EXPERT_BIAS = 1, 2

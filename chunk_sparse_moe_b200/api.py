@@ -87,9 +87,9 @@ def route(x: torch.Tensor, W_r: torch.Tensor, gamma: torch.Tensor, eps: float,
 
 
 def residual_layernorm(y: torch.Tensor, x: torch.Tensor, ln_gamma: torch.Tensor,
-                       ln_beta: torch.Tensor, eps: float = 1e-5,
+                       ln_beta: Optional[torch.Tensor], eps: float = 1e-5,
                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """out [T, d_h] = LayerNorm(y + x) over d_h (scale ln_gamma, shift ln_beta, fp32)."""
+    """out [T, d_h] = LayerNorm(y + x) over d_h (scale ln_gamma, shift ln_beta or none, fp32)."""
     T, d_h = x.shape
     if out is None:
         out = torch.empty_like(x)
@@ -114,9 +114,9 @@ def chunk_union(gates: torch.Tensor, n: int):
 
 
 def workspace_bytes(T: int, d_h: int, E: int, d_e: int, n: int, dtype: torch.dtype,
-                    with_router: bool) -> int:
-    return int(lib.blockffn_forward_workspace_bytes(T, d_h, E, d_e, n, _DT[dtype],
-                                                    1 if with_router else 0))
+                    with_router: bool, with_bias: bool = False) -> int:
+    flags = (_lib.WS_ROUTER if with_router else 0) | (_lib.WS_EXPERT_BIAS if with_bias else 0)
+    return int(lib.blockffn_forward_workspace_bytes(T, d_h, E, d_e, n, _DT[dtype], flags))
 
 
 class Workspace:
@@ -136,8 +136,9 @@ class Workspace:
                "blockffn_workspace_reset")
 
     @classmethod
-    def for_shapes(cls, T, d_h, E, d_e, n, dtype, with_router, device=None) -> "Workspace":
-        nb = workspace_bytes(T, d_h, E, d_e, n, dtype, with_router)
+    def for_shapes(cls, T, d_h, E, d_e, n, dtype, with_router, device=None,
+                   with_bias: bool = False) -> "Workspace":
+        nb = workspace_bytes(T, d_h, E, d_e, n, dtype, with_router, with_bias)
         if nb == 0:
             raise BlockFFNError(_lib.ERR_INVALID_ARG, "blockffn_forward_workspace_bytes")
         return cls(nb, device)
@@ -147,21 +148,33 @@ def forward(x: torch.Tensor, W_in: torch.Tensor, W_out: torch.Tensor, n: int,
             gates: Optional[torch.Tensor] = None, W_r: Optional[torch.Tensor] = None,
             b_r: Optional[torch.Tensor] = None, gamma: Optional[torch.Tensor] = None,
             eps: float = 2.0 ** -23, y: Optional[torch.Tensor] = None,
-            workspace: Optional[Workspace] = None, union=None) -> torch.Tensor:
-    """y [T, d_h] = sum over each chunk's union experts of gate * W_out_e Swish(W_in_e x).
+            workspace: Optional[Workspace] = None, union=None,
+            b_in: Optional[torch.Tensor] = None, b_out: Optional[torch.Tensor] = None,
+            ln_weight: Optional[torch.Tensor] = None, ln_bias: Optional[torch.Tensor] = None,
+            ln_eps: float = 1e-5) -> torch.Tensor:
+    """y [T, d_h] = sum over each chunk's union experts of
+    gate * (W_out_e Swish(W_in_e x + b_in_e) + b_out_e), then LayerNorm(y + x) when
+    ``ln_weight`` is given.
 
     ``union``: optional (counts, idx, tmask) as ``chunk_union`` returns them for
-    these gates and n; the forward then uses them instead of forming the union."""
+    these gates and n; the forward then uses them instead of forming the union.
+    ``b_in`` [E, d_e], ``b_out`` [E, d_h], ``ln_weight``/``ln_bias`` [d_h]: fp32,
+    optional (a workspace for ``b_out`` is sized with ``with_bias=True``)."""
     T, d_h = x.shape
     E, d_e, _ = W_in.shape
     if y is None:
         y = torch.empty((T, d_h), dtype=x.dtype, device=x.device)
     if workspace is None:
-        workspace = Workspace.for_shapes(T, d_h, E, d_e, n, x.dtype, gates is None, x.device)
+        workspace = Workspace.for_shapes(T, d_h, E, d_e, n, x.dtype, gates is None, x.device,
+                                         with_bias=b_out is not None)
     counts, idx, tmask = union if union is not None else (None, None, None)
+    opts = None
+    if b_in is not None or b_out is not None or ln_weight is not None:
+        opts = ctypes.byref(_lib.LayerOpts(_ptr(b_in), _ptr(b_out), _ptr(ln_weight), _ptr(ln_bias),
+                                           float(ln_eps)))
     st = lib.blockffn_forward(_ptr(x), _ptr(gates), _ptr(W_r), _ptr(b_r), _ptr(gamma), float(eps),
                               _ptr(counts), _ptr(idx), _ptr(tmask),
-                              _ptr(W_in), _ptr(W_out), T, d_h, E, d_e, n, _dtype_code(x),
+                              _ptr(W_in), _ptr(W_out), T, d_h, E, d_e, n, _dtype_code(x), opts,
                               _ptr(y), workspace.buf.data_ptr(), workspace.nbytes, _stream())
     _check(st, "blockffn_forward")
     return y

@@ -140,6 +140,8 @@ struct Layout {
     Path path;
     size_t ctl, counts, offsets, idx, tmask, pair_ce, gcounts, goffsets, gpair, gates;
     size_t readyA, cntB, partB, hbuf;
+    size_t ybias;        // group path with fc2 biases: [T, d_h] fp32 per-token bias sums
+    size_t lnstats;      // single-chunk path: [RT*4][32] (mean, M2) of the LayerNorm slices
     size_t total;
     int C;               // chunks
     int N;               // tokens per MMA
@@ -169,7 +171,8 @@ int decode_grid(int C, int d_h, int E, int G) {
     return 4 * ncl;
 }
 
-void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_router, int G, Layout& L) {
+void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_router, bool with_bias, int G,
+                 Layout& L) {
     L.C = (T + n - 1) / n;
     L.MT = bf16 ? d_e / 128 : 1;
     L.RT = bf16 ? d_h / 128 : 1;
@@ -183,7 +186,7 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         return o;
     };
     L.ctl = L.counts = L.offsets = L.idx = L.tmask = L.pair_ce = L.gcounts = L.goffsets = L.gpair = 0;
-    L.gates = L.readyA = L.cntB = L.partB = L.hbuf = 0;
+    L.gates = L.readyA = L.cntB = L.partB = L.hbuf = L.ybias = L.lnstats = 0;
     L.NG = L.NT = L.NGr = 0;
     const size_t C = (size_t)L.C;
     L.ctl = take(sizeof(Ctl));
@@ -203,6 +206,7 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         L.Pmax = E;
         L.readyA = take(2 * (size_t)E * 4);
         L.hbuf = take((size_t)E * L.N * d_e * 2);
+        L.lnstats = take((size_t)L.RT * 4 * 32 * 8);
     } else {
         // groups of whole chunks, N = 128 tokens per MMA for short inputs, else 256
         L.N = T <= 128 ? 128 : 256;
@@ -221,6 +225,7 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         L.cntB = take(2 * NGr * L.RT * 4);
         L.partB = take((size_t)G * 2 * L.N * 128 * 4);
         L.hbuf = take(Pm * L.N * d_e * 2);
+        if (with_bias) L.ybias = take((size_t)T * d_h * 4);
     }
     L.total = off;
 }
@@ -303,7 +308,7 @@ blockffn_status blockffn_residual_layernorm(const void* y, const void* x, const 
     if (T < 0 || d_h < 1) return fail(BLOCKFFN_ERR_INVALID_ARG, "bad shape (T = %d, d_h = %d)", T, d_h);
     if (!(eps >= 0.f) || !std::isfinite(eps)) return fail(BLOCKFFN_ERR_INVALID_ARG, "eps must be finite and >= 0");
     if (T == 0) return BLOCKFFN_OK;
-    if (!y || !x || !ln_gamma || !ln_beta || !out) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
+    if (!y || !x || !ln_gamma || !out) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
     cudaError_t e = launch_residual_layernorm(y, x, ln_gamma, ln_beta, eps, T, d_h, dt == BLOCKFFN_BF16, out,
                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "residual layernorm launch");
@@ -318,13 +323,14 @@ blockffn_status blockffn_chunk_union(const float* gates, int T, int E, int n, in
     return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "chunk_union launch");
 }
 
-size_t blockffn_forward_workspace_bytes(int T, int d_h, int E, int d_e, int n, blockffn_dtype dt,
-                                        int with_router) {
+size_t blockffn_forward_workspace_bytes(int T, int d_h, int E, int d_e, int n, blockffn_dtype dt, int flags) {
     if (check_shapes(T, d_h, E, d_e, n, dt) != BLOCKFFN_OK) return 0;
+    if ((flags & ~(BLOCKFFN_WS_ROUTER | BLOCKFFN_WS_EXPERT_BIAS)) != 0) return 0;
     const int G = num_sms_current();
     if (G <= 0) return 0;
     Layout L;
-    make_layout(T, d_h, E, d_e, n, dt == BLOCKFFN_BF16, with_router != 0, G, L);
+    make_layout(T, d_h, E, d_e, n, dt == BLOCKFFN_BF16, (flags & BLOCKFFN_WS_ROUTER) != 0,
+                (flags & BLOCKFFN_WS_EXPERT_BIAS) != 0, G, L);
     return L.total;
 }
 
@@ -338,8 +344,8 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
                                  const float* b_r, const float* gamma, float eps,
                                  const int32_t* counts, const int32_t* idx, const uint32_t* tmask,
                                  const void* W_in, const void* W_out, int T, int d_h, int E,
-                                 int d_e, int n, blockffn_dtype dt, void* y, void* workspace,
-                                 size_t ws_bytes, void* stream) {
+                                 int d_e, int n, blockffn_dtype dt, const blockffn_layer_opts* opts,
+                                 void* y, void* workspace, size_t ws_bytes, void* stream) {
     blockffn_status st = check_shapes(T, d_h, E, d_e, n, dt);
     if (st != BLOCKFFN_OK) return st;
     if (T == 0) return BLOCKFFN_OK;   // nothing to compute (empty tensors may be NULL)
@@ -359,6 +365,16 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         return fail(BLOCKFFN_ERR_INVALID_ARG, "pass either gates or router weights, not both");
     }
     if (!x || !W_in || !W_out || !y || !workspace) return fail(BLOCKFFN_ERR_INVALID_ARG, "null pointer");
+    const float* b_in = opts ? opts->b_in : nullptr;
+    const float* b_out = opts ? opts->b_out : nullptr;
+    const float* ln_w = opts ? opts->ln_weight : nullptr;
+    const float* ln_b = (opts && ln_w) ? opts->ln_bias : nullptr;
+    const float ln_eps = opts ? opts->ln_eps : 0.f;
+    if (ln_w && (!(ln_eps >= 0.f) || !std::isfinite(ln_eps)))
+        return fail(BLOCKFFN_ERR_INVALID_ARG, "ln_eps must be finite and >= 0");
+    if ((b_in && !aligned16(b_in)) || (b_out && !aligned16(b_out)) || (ln_w && !aligned16(ln_w)) ||
+        (ln_b && !aligned16(ln_b)))
+        return fail(BLOCKFFN_ERR_INVALID_ARG, "bias and LayerNorm pointers must be 16-byte aligned");
     if (!aligned16(x) || !aligned16(W_in) || !aligned16(W_out) || !aligned16(y) ||
         !aligned16(workspace) || (gates && !aligned16(gates)) || (W_r && !aligned16(W_r)) ||
         (gamma && !aligned16(gamma)) || (b_r && !aligned16(b_r)) || (counts && !aligned16(counts)) ||
@@ -367,10 +383,19 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     const int G = num_sms_current();
     if (G <= 0) return fail(BLOCKFFN_ERR_CUDA, "no current CUDA device");
     const bool bf16 = dt == BLOCKFFN_BF16;
+    const bool with_bias = b_out != nullptr;
     Layout L;
-    make_layout(T, d_h, E, d_e, n, bf16, routed, G, L);
+    make_layout(T, d_h, E, d_e, n, bf16, routed, with_bias, G, L);
     if (ws_bytes < L.total)
-        return fail(BLOCKFFN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, L.total);
+        return fail(BLOCKFFN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed%s", ws_bytes, L.total,
+                    with_bias ? " (fc2 biases: size it with BLOCKFFN_WS_EXPERT_BIAS)" : "");
+    // the LayerNorm as its own kernel after the forward, rewriting y in place
+    auto closing_layernorm = [&]() -> blockffn_status {
+        if (!ln_w) return BLOCKFFN_OK;
+        cudaError_t e2 = launch_residual_layernorm(y, x, ln_w, ln_b, ln_eps, T, d_h, bf16, y,
+                                                   static_cast<cudaStream_t>(stream));
+        return e2 == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e2, "residual layernorm launch");
+    };
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
     Ctl* ctl = reinterpret_cast<Ctl*>(ws + L.ctl);
@@ -396,10 +421,11 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
                                     d_h, 4, s);
         if (e != cudaSuccess) return cuda_fail(e, "union launch");
         e = launch_forward_f32(static_cast<const float*>(x), g, static_cast<const float*>(W_in),
-                               static_cast<const float*>(W_out), t_counts, offsets, pair_ce, t_tmask, ctl,
-                               reinterpret_cast<float*>(ws + L.hbuf), T, d_h, E, d_e, n,
+                               static_cast<const float*>(W_out), b_in, b_out, t_counts, offsets, pair_ce,
+                               t_tmask, ctl, reinterpret_cast<float*>(ws + L.hbuf), T, d_h, E, d_e, n,
                                static_cast<float*>(y), G, s);
-        return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "fp32 forward launch");
+        if (e != cudaSuccess) return cuda_fail(e, "fp32 forward launch");
+        return closing_layernorm();
     }
 
     if (L.path == Path::Decode) {
@@ -422,6 +448,16 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
         da.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
         da.ctl = ctl;
+        da.x = static_cast<const __nv_bfloat16*>(x);
+        da.b_in = b_in;
+        da.b_out = b_out;
+        // the LayerNorm in the kernel's last step when every row tile of y has a
+        // cluster of its own, else as a kernel of its own afterwards
+        const bool ln_fused = ln_w != nullptr && L.RT <= Gd / 4;
+        da.ln_w = ln_fused ? ln_w : nullptr;
+        da.ln_b = ln_fused ? ln_b : nullptr;
+        da.ln_eps = ln_eps;
+        da.ln_stats = reinterpret_cast<float2*>(ws + L.lnstats);
         da.T = T;
         da.d_h = d_h;
         da.E = E;
@@ -433,11 +469,12 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.skip_unit = g_skip_flag.load();
         da.wait_ns = g_wait_ns.load();
         da.trace = g_trace.load();
-        da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1, Gd});
+        da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1, Gd, with_bias ? 1 : 0});
         // A cluster launch cannot also be cooperative; the grid is sized to the
         // clusters that can be resident at once, and every wait is bounded.
         e = launch_forward_decode(da, dmaps, Gd, s);
-        return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "single-chunk forward launch");
+        if (e != cudaSuccess) return cuda_fail(e, "single-chunk forward launch");
+        return ln_fused ? BLOCKFFN_OK : closing_layernorm();
     }
 
     // several chunks (or one the single-chunk kernel cannot take): group tables,
@@ -448,6 +485,11 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     e = launch_group_plan(g, T, E, n, t_counts, t_idx, t_tmask, !tables, ctl, L.NG, L.NGr, gcounts, goffsets,
                           gpair, static_cast<__nv_bfloat16*>(y), d_h, s);
     if (e != cudaSuccess) return cuda_fail(e, "group plan launch");
+    float* ybias = with_bias ? reinterpret_cast<float*>(ws + L.ybias) : nullptr;
+    if (with_bias) {
+        e = launch_expert_bias_sum(g, t_counts, t_idx, t_tmask, ctl, b_out, T, d_h, E, n, ybias, s);
+        if (e != cudaSuccess) return cuda_fail(e, "expert bias launch");
+    }
     CUtensorMap maps[5];
     // expert-out partial tiles [blocks][2 slots][N/4 token quads][128 rows x 4 tokens]
     // fp32, seen as lines of 512 floats; a box is 32 rows of every token quad
@@ -471,6 +513,8 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.cnt_b_len = (long long)L.NGr * L.RT;
     a.ctl = ctl;
     a.y = static_cast<__nv_bfloat16*>(y);
+    a.b_in = b_in;
+    a.ybias = ybias;
     a.T = T;
     a.d_h = d_h;
     a.E = E;
@@ -485,10 +529,11 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.KBe = L.KBe;
     a.skip_flag_unit = g_skip_flag.load();
     a.wait_ns = g_wait_ns.load();
-    a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2, G});
+    a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2, G, with_bias ? 1 : 0});
     a.trace = g_trace.load();
     e = launch_forward_group(a, maps, G, s);
-    return e == cudaSuccess ? BLOCKFFN_OK : cuda_fail(e, "group forward launch");
+    if (e != cudaSuccess) return cuda_fail(e, "group forward launch");
+    return closing_layernorm();
 }
 
 // ------------------------------------------------------------------------
@@ -575,6 +620,13 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     da.hbuf = reinterpret_cast<__nv_bfloat16*>(scratch + off_h);
     da.readyA = reinterpret_cast<uint32_t*>(scratch + off_ready);
     da.ctl = reinterpret_cast<Ctl*>(scratch);
+    da.x = static_cast<const __nv_bfloat16*>(x);
+    da.b_in = nullptr;
+    da.b_out = nullptr;
+    da.ln_w = nullptr;
+    da.ln_b = nullptr;
+    da.ln_eps = 0.f;
+    da.ln_stats = nullptr;
     da.T = T;
     da.d_h = d_h;
     da.E = E;

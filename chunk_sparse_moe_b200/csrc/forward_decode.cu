@@ -33,6 +33,20 @@
 // block of rank q, which adds the 4 contributions in rank order (a fixed order)
 // and writes those 32 rows of y.
 //
+// Optional parts of the layer (the experts' nn.Linear biases, Router
+// Architecture Setup; the closing LayerNorm, Full BlockFFN Layer with Combined
+// Losses).  The fc1 bias of an accumulator row is added before Swish.  The
+// summing warp of a row slice adds, before the four partials, the gated fc2
+// biases of its rows: sum over the union, ascending, of bit_t ? g[t,e] b_out[e,i]
+// : 0 (computed while the expert-out MMAs run).  With a LayerNorm, v = sum + x
+// stays in fp32: each summing warp publishes its 32-row slice's per-token mean
+// and sum of squared deviations, counts the slice in (release), waits (bounded)
+// until every slice of y is counted in, forms each token's mean and variance from
+// the slices in slice order (the two-level decomposition of the variance: exact,
+// and in a fixed order), and stores ln_w * (v - mean) / sqrt(var + eps) + ln_b.
+// That needs every row tile of y summed by a cluster of its own (one slice per
+// summing warp); the host otherwise runs the LayerNorm as a following kernel.
+//
 // Roles (224 threads): warp 0 TMA producer (one lane), warp 1 MMA issuer (the
 // whole warp runs its loops and waits, one elected lane issues), warp 2 TMEM
 // owner and h' loader, warps 3-6 epilogue.  Every wait is bounded; a timeout
@@ -214,6 +228,37 @@ __device__ __forceinline__ RsWork rs_work(int G, int P, int MT, int KPe, int RT)
     return w;
 }
 
+// Sums over the warp's 32 lanes of one value per token, scattered: on return
+// lane j holds the sum over the lanes of v[j % N] (v is consumed).  A fixed
+// butterfly, so the sums do not depend on timing.
+template <int N>
+__device__ __forceinline__ float rs_warp_sum_scatter(float (&v)[N]) {
+    const int lane = threadIdx.x & 31;
+    if constexpr (N == 16) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 16);
+    }
+#pragma unroll
+    for (int off = N / 2; off >= 1; off >>= 1) {
+        const bool up = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+            const float send = up ? v[i] : v[i + off];
+            const float keep = up ? v[i + off] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return v[0];
+}
+
+// The same total in every lane (an xor butterfly: every lane adds the same two
+// values at every level, so all lanes hold the same bits).
+__device__ __forceinline__ float rs_warp_allsum(float v) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
 template <int N>
 __global__ void __launch_bounds__(kRsThreads, 1)
 union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_win,
@@ -280,7 +325,11 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const unsigned long long tk = atomicAdd(&a.ctl->ticket, 1ull);
         const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
         const uint32_t ep0 = (uint32_t)(tk / gridDim.x);
-        if (blockIdx.x == 0) a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;   // the next launch's counter
+        if (blockIdx.x == 0) {
+            // the next launch's counters
+            a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;
+            a.ctl->ln_cnt[(ep0 & 1u) ^ 1u] = 0u;
+        }
         sh.epoch = ep0;
         const bool key_ok = key0 == 0ull || key0 == a.shape_key;
         if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
@@ -607,8 +656,30 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // meet the same named barriers.
         bool failed = abort_at_start;
         if (P == 0 && blockIdx.x == 0 && !failed) {
-            // empty union: y is all zeros
-            for (size_t k2 = et; k2 < (size_t)nt * a.d_h; k2 += 128) a.y[k2] = __float2bfloat16_rn(0.f);
+            if (a.ln_w == nullptr) {
+                // empty union: y is all zeros
+                for (size_t k2 = et; k2 < (size_t)nt * a.d_h; k2 += 128) a.y[k2] = __float2bfloat16_rn(0.f);
+            } else {
+                // empty union: the expert sum is zero, y = LayerNorm(x); warp w
+                // takes tokens w, w + 4, ... (two passes over the row, then the store)
+                for (int t = warp - 3; t < nt; t += 4) {
+                    const __nv_bfloat16* xr = a.x + (size_t)t * a.d_h;
+                    float sm = 0.f;
+                    for (int k2 = lane; k2 < a.d_h; k2 += 32) sm += __bfloat162float(xr[k2]);
+                    const float mu = rs_warp_allsum(sm) / (float)a.d_h;
+                    float q = 0.f;
+                    for (int k2 = lane; k2 < a.d_h; k2 += 32) {
+                        const float dv = __bfloat162float(xr[k2]) - mu;
+                        q = fmaf(dv, dv, q);
+                    }
+                    const float rstd = 1.0f / sqrtf(rs_warp_allsum(q) / (float)a.d_h + a.ln_eps);
+                    for (int k2 = lane; k2 < a.d_h; k2 += 32) {
+                        const float o = a.ln_w[k2] * ((__bfloat162float(xr[k2]) - mu) * rstd) +
+                                        (a.ln_b != nullptr ? a.ln_b[k2] : 0.f);
+                        a.y[(size_t)t * a.d_h + k2] = __float2bfloat16_rn(o);
+                    }
+                }
+            }
         }
         // ---- A units: each block finishes its half of the tokens
         const uint32_t peer = (uint32_t)(wk.cr ^ 1);
@@ -624,6 +695,8 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             // stage the unit's gates now: the accumulator wait hides their latency,
             // and the activation loop below then reads shared memory only
             if (et < 32) sh.s_gate[b][et] = a.gates[(size_t)min(et, nt - 1) * a.E + e];
+            // this accumulator row's fc1 bias (0 without biases)
+            const float bin = a.b_in != nullptr ? __ldg(a.b_in + (size_t)e * a.d_e + mt * 128 + row) : 0.f;
             if (et == 0) {
                 // the peer's partial for this block's half of unit ua lands in buffer b
                 mbar_arrive_expect_tx(&sh.recvA[b], (uint32_t)(NH * 128 * 4));
@@ -704,7 +777,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 __nv_bfloat16 hb[NH];
 #pragma unroll
                 for (int tl = 0; tl < NH; ++tl)
-                    hb[tl] = __float2bfloat16_rn(((bits >> tl) & 1u) ? gv[tl] * rs_swish(z[tl]) : 0.f);
+                    hb[tl] = __float2bfloat16_rn(((bits >> tl) & 1u) ? gv[tl] * rs_swish(z[tl] + bin) : 0.f);
                 __nv_bfloat16* stg = hstage + row;
 #pragma unroll
                 for (int tl = 0; tl < NH; ++tl) stg[tl * 128] = hb[tl];
@@ -746,6 +819,22 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 const int rt = wk.rt0 + k * wk.rtstep;
                 const int ab = k & 1;
                 uint32_t r[32];
+                // the summing warp's gated fc2 bias sums of its 32 rows, formed while
+                // the expert-out MMAs run: lane = row, bacc[t] for token t
+                float bacc[N];
+#pragma unroll
+                for (int t = 0; t < N; ++t) bacc[t] = 0.f;
+                if (a.b_out != nullptr && qd == wk.cr) {
+                    const float* bo = a.b_out + rt * 128 + wk.cr * 32 + lane;
+                    for (int s2 = 0; s2 < P; ++s2) {
+                        const int e = sh.s_pair_e[s2];
+                        const uint32_t bits = sh.s_tmask[e];
+                        const float bv = __ldg(bo + (size_t)e * a.d_h);
+                        const float gl = (lane < nt && ((bits >> lane) & 1u)) ? a.gates[(size_t)lane * a.E + e] : 0.f;
+#pragma unroll
+                        for (int t = 0; t < N; ++t) bacc[t] = fmaf(__shfl_sync(0xffffffffu, gl, t), bv, bacc[t]);
+                    }
+                }
                 if (nBt > 0) {
                     if (et == 0)
                         sh.ep_okB[0] = wait_bar(&sh.accB_full[ab], (uint32_t)((k >> 1) & 1), limit, &sh.abort, a.ctl,
@@ -796,10 +885,10 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         if (ok) sh.pendB = -1;
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
+                    float acc[N];
                     if (ok) {
-                        float acc[N];
 #pragma unroll
-                        for (int t = 0; t < N; ++t) acc[t] = 0.f;
+                        for (int t = 0; t < N; ++t) acc[t] = bacc[t];
 #pragma unroll
                         for (int q = 0; q < kRsCluster; ++q) {
                             if (q == wk.cr) {
@@ -817,6 +906,57 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                                 }
                             }
                         }
+                        if (a.ln_w != nullptr) {
+                            // LayerNorm(sum + x): this slice's statistics out, every
+                            // slice's in (see the file's header)
+                            const int i = rt * 128 + wk.cr * 32 + lane;   // this lane's row
+#pragma unroll
+                            for (int t = 0; t < N; ++t)
+                                if (t < nt) acc[t] += __bfloat162float(a.x[(size_t)t * a.d_h + i]);
+                            float tmp[N];
+#pragma unroll
+                            for (int t = 0; t < N; ++t) tmp[t] = acc[t];
+                            const float mloc = rs_warp_sum_scatter<N>(tmp) * (1.0f / 32.0f);
+#pragma unroll
+                            for (int t = 0; t < N; ++t) {
+                                const float dv = acc[t] - __shfl_sync(0xffffffffu, mloc, t);
+                                tmp[t] = dv * dv;
+                            }
+                            const float m2loc = rs_warp_sum_scatter<N>(tmp);
+                            const int nsl = a.RT * 4;                     // 32-row slices of y
+                            float2* stats = a.ln_stats;
+                            stats[(size_t)(rt * 4 + wk.cr) * 32 + lane] = make_float2(mloc, m2loc);
+                            __syncwarp();
+                            if (lane == 0) {
+                                __threadfence();
+                                red_release_add_gpu(&a.ctl->ln_cnt[par], 1u);
+                                ok = wait_count(&a.ctl->ln_cnt[par], (uint32_t)nsl, limit_peer, &sh.abort, a.ctl,
+                                                kWaitPeers) ? 1 : 0;
+                                __threadfence();
+                            }
+                            ok = __shfl_sync(0xffffffffu, ok, 0);
+                            if (ok) {
+                                // lane t: token t's mean over the slices, then its sum of
+                                // squared deviations, both in slice order
+                                float mu = 0.f;
+                                for (int j = 0; j < nsl; ++j) mu += __ldcg(&stats[(size_t)j * 32 + lane]).x;
+                                mu /= (float)nsl;
+                                float m2 = 0.f;
+                                for (int j = 0; j < nsl; ++j) {
+                                    const float2 st = __ldcg(&stats[(size_t)j * 32 + lane]);
+                                    const float dm = st.x - mu;
+                                    m2 += st.y + 32.f * dm * dm;
+                                }
+                                const float rstd = 1.0f / sqrtf(m2 / (float)a.d_h + a.ln_eps);
+                                const float wgt = a.ln_w[i], sft = a.ln_b != nullptr ? a.ln_b[i] : 0.f;
+#pragma unroll
+                                for (int t = 0; t < N; ++t)
+                                    acc[t] = wgt * ((acc[t] - __shfl_sync(0xffffffffu, mu, t)) *
+                                                    __shfl_sync(0xffffffffu, rstd, t)) + sft;
+                            }
+                        }
+                    }
+                    if (ok) {
                         // rows 32*cr.. of y for all tokens: staged [N tokens][32 rows]
                         // bf16, then one TMA store (rows past T are clipped)
                         if (k > 0 && lane == 0) bulk_wait_group_read0();   // staging free again

@@ -18,9 +18,12 @@
 //
 // Work.  For every group G and expert e of its set (a "pair" p):
 //   expert-in  : h^T[d_e, N]  = W_in_e[d_e, d_h] . x_G^T[d_h, N]           (A units)
-//                h'[j, :]     = bit_j ? g[t_j, e] * Swish(h[j, :]) : 0      (epilogue)
+//                h'[j, :]     = bit_j ? g[t_j, e] * Swish(h[j, :] + b_in_e) : 0   (epilogue)
 //   expert-out : y_G^T[d_h,N] = sum_{e in U_G, ascending} W_out_e . h'_e^T  (B units)
-// bit_j is token t_j's bit in its chunk's token mask (the chunk union tables).
+//                y[t, :]     += ybias[t, :]   (the gated fc2 biases, expert_bias.cu)
+// bit_j is token t_j's bit in its chunk's token mask (the chunk union tables);
+// the biases (the experts' nn.Linear biases, Router Architecture Setup) are
+// optional.
 //
 // Schedule.  One persistent block per SM (cooperative launch: all resident).  The
 // A work is dealt out in whole units (a pair's 128-row tile of W_in_e over all of
@@ -33,11 +36,12 @@
 // with a bounded spin, until the block owning the expert-in unit it reads has
 // written that unit's h'.
 //
-// Roles (224 threads): warp 0 issues the weight-tile TMA loads, warp 1 issues
+// Roles (352 threads): warp 0 issues the weight-tile TMA loads, warp 1 issues
 // the MMAs (the whole warp runs the loop, one elected lane issues), warp 2 owns
 // TMEM and issues the activation-tile TMA loads (x, or h' once its flag is set),
-// warps 3-6 drain the accumulators (TMEM -> registers, 32 columns at a time) and
-// do the split reductions, Swish, gate, mask and stores.
+// warps 3-10 drain the accumulators (TMEM -> registers, 32 columns at a time, two
+// warp groups on alternate column slices) and do the split reductions, Swish,
+// gate, mask and stores.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -607,11 +611,16 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     if (!last) {
                         ring4[off] = acc;
                     } else {
-                        __nv_bfloat16* ycol = a.y + (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + r0 + rr;
+                        const size_t col = (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + r0 + rr;
+                        __nv_bfloat16* ycol = a.y + col;
                         const float z[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
-                            if (4 * kq + u < nvalid) ycol[(size_t)(4 * kq + u) * a.d_h] = __float2bfloat16_rn(z[u]);
+                            if (4 * kq + u < nvalid) {
+                                const size_t o = (size_t)(4 * kq + u) * a.d_h;
+                                const float yb = a.ybias != nullptr ? __ldg(a.ybias + col + o) : 0.f;
+                                ycol[o] = __float2bfloat16_rn(z[u] + yb);
+                            }
                     }
                 }
                 named_bar_sync(1, kGrEpi);   // the ring is read; the next batch may land
@@ -698,6 +707,9 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 __nv_bfloat16* dst;
                 size_t ld;
                 int ntok;
+                // fc1 bias of this accumulator row (expert-in units), or 0
+                const float bin = (sg.kind == 0 && a.b_in != nullptr)
+                                      ? __ldg(a.b_in + (size_t)sg.e * a.d_e + sg.mt * 128 + row) : 0.f;
                 if (sg.kind == 0) {
                     dst = a.hbuf + (size_t)sg.p * N * a.d_e + sg.mt * 128;
                     ld = (size_t)a.d_e;
@@ -732,9 +744,18 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                         }
 #pragma unroll
                         for (int u = 0; u < 32; ++u) {
-                            const float h = ((bits >> u) & 1u) ? gv[u] * gr_swish(__uint_as_float(r[u])) : 0.f;
+                            const float h =
+                                ((bits >> u) & 1u) ? gv[u] * gr_swish(__uint_as_float(r[u]) + bin) : 0.f;
                             hb[u] = __float2bfloat16_rn(h);
                         }
+                    } else if (a.ybias != nullptr) {
+                        // the tokens' fc2 bias sums of this row (fp32, added before rounding)
+                        float yb[32];
+                        const float* ybc = a.ybias + (size_t)(sg.g * a.NT + c0) * a.d_h + sg.rt * 128 + row;
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) yb[u] = c0 + u < ntok ? __ldg(ybc + (size_t)u * a.d_h) : 0.f;
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) hb[u] = __float2bfloat16_rn(__uint_as_float(r[u]) + yb[u]);
                     } else {
 #pragma unroll
                         for (int u = 0; u < 32; ++u) hb[u] = __float2bfloat16_rn(__uint_as_float(r[u]));

@@ -39,11 +39,19 @@ cudaError_t launch_group_plan(const float* gates, int T, int E, int n, int32_t* 
                               int32_t* gcounts, int32_t* goffsets, int32_t* gpair, __nv_bfloat16* y,
                               int d_h, cudaStream_t s);
 
+// b_in [E, d_e] and b_out [E, d_h] fp32 expert biases, or nullptr
 cudaError_t launch_forward_f32(const float* x, const float* gates, const float* W_in,
-                               const float* W_out, const int32_t* counts, const int32_t* offsets,
+                               const float* W_out, const float* b_in, const float* b_out,
+                               const int32_t* counts, const int32_t* offsets,
                                const int32_t* pair_ce, const uint32_t* tmask, const Ctl* ctl,
                                float* hbuf, int T, int d_h, int E, int d_e, int n, float* y,
                                int num_sms, cudaStream_t s);
+
+// ybias[t, :] = sum over the union of t's chunk (ascending) of the gate-masked
+// fc2 biases, bit_t ? g[t,e] b_out[e,:] : 0, fp32 [T, d_h] (expert_bias.cu)
+cudaError_t launch_expert_bias_sum(const float* gates, const int32_t* counts, const int32_t* idx,
+                                   const uint32_t* tmask, const Ctl* ctl, const float* b_out, int T,
+                                   int d_h, int E, int n, float* ybias, cudaStream_t s);
 
 // Arguments of the multi-chunk group forward (forward_group.cu).
 struct GrArgs {
@@ -60,6 +68,8 @@ struct GrArgs {
     long long cnt_b_len;      // NGr*RT
     Ctl* ctl;
     __nv_bfloat16* y;         // [T, d_h]
+    const float* b_in;        // [E, d_e] fc1 biases, or nullptr
+    const float* ybias;       // [T, d_h] per-token fc2 bias sums (expert_bias.cu), or nullptr
     int T, d_h, E, d_e, n;
     int N;     // tokens per MMA: 128 or 256
     int NT;    // tokens per group: (N / n) * n
@@ -90,6 +100,15 @@ struct DcArgs {
     __nv_bfloat16* hbuf;      // [E slots][N][d_e] gated activations h'
     uint32_t* readyA;         // [2][E] halves of an expert slot written, by launch parity
     Ctl* ctl;
+    const __nv_bfloat16* x;   // [T, d_h] (the LayerNorm's residual)
+    const float* b_in;        // [E, d_e] fc1 biases, or nullptr
+    const float* b_out;       // [E, d_h] fc2 biases, or nullptr
+    // LayerNorm(sum + x) in the last step when ln_w != nullptr (every row tile of
+    // y then has a cluster of its own: RT <= clusters); ln_b may be nullptr
+    const float* ln_w;
+    const float* ln_b;
+    float ln_eps;
+    float2* ln_stats;         // [RT*4 slices][32 tokens] (mean, M2) of a 32-row slice
     int T, d_h, E, d_e, n, N;
     int KB;    // d_h / 64
     int RT;    // d_h / 128

@@ -5,7 +5,7 @@
 // input to the expert sum and normalises the result with nn.LayerNorm over the
 // hidden dimension: per-feature scale and shift, population variance).
 //
-// One block per token row.  v = y + x in fp32; each thread walks k = tid,
+// One block per token row (ln_beta may be null: no shift).  v = y + x in fp32; each thread walks k = tid,
 // tid + 256, ... in ascending order, the 256 partial sums meet in a fixed tree
 // (a warp butterfly, then the 8 warps' sums in warp order), so the statistics do
 // not depend on timing.  The variance is a second pass around the mean; a third
@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kLnThreads) residual_layernorm_kernel(
     const float rstd = 1.0f / sqrtf(var + eps);
     for (int k = threadIdx.x; k < d_h; k += kLnThreads) {
         const float v = ln_f32(yr[k]) + ln_f32(xr[k]);
-        ln_store(o + k, ln_gamma[k] * ((v - mu) * rstd) + ln_beta[k]);
+        ln_store(o + k, ln_gamma[k] * ((v - mu) * rstd) + (ln_beta != nullptr ? ln_beta[k] : 0.f));
     }
 }
 

@@ -8,8 +8,10 @@
  *
  *   route:  g[t,:] = RMSNorm(ReLU(W_r x_t + b_r))          over the E experts
  *   union:  U_c    = { e : g[t,e] != 0 for some t in chunk c }, chunks of n tokens
- *   expert: o_e(x) = W_out_e Swish(W_in_e x)                non-gated, d_e << d_h
+ *   expert: o_e(x) = W_out_e Swish(W_in_e x + b_in_e) + b_out_e   non-gated, d_e << d_h
+ *                    (the biases are optional)
  *   output: y[t,:] = sum_{e in U_c, ascending} [g[t,e] != 0] g[t,e] o_e(x_t)
+ *           optionally followed by y <- LayerNorm(y + x) over d_h
  *
  * Only the union experts run, each over every token of the chunk as one small
  * dense GEMM pair; tokens whose own gate is zero are masked after computing.
@@ -119,7 +121,8 @@ blockffn_status blockffn_chunk_union(const float* gates, int T, int E, int n,
  * Full BlockFFN Layer with Combined Losses (the expert sum plus the input, through
  * nn.LayerNorm(hidden_dim); its default eps is 1e-5).
  * y, x, out [T, d_h] in dtype dt (out may alias y or x: every element is read
- * before it is written); ln_gamma, ln_beta [d_h] fp32; eps finite and >= 0.
+ * before it is written); ln_gamma [d_h] fp32; ln_beta [d_h] fp32 or NULL (no
+ * shift); eps finite and >= 0.
  * Arithmetic: fp32 from the dt inputs, the sums in a fixed order, out rounded once
  * to dt.  Stream-ordered; launched as a programmatic dependent of the preceding
  * kernel (it reads nothing before that kernel has completed).
@@ -129,12 +132,45 @@ blockffn_status blockffn_residual_layernorm(const void* y, const void* x, const 
                                            blockffn_dtype dt, void* out, void* stream);
 
 /*
+ * blockffn_layer_opts -- the optional parts of the layer around the expert sum,
+ * passed to blockffn_forward (a NULL pointer there means none of them).
+ * Pages: "BlockFFN: Sparse Mixture-of-Experts Optimized for End-Device Deployment",
+ * Router Architecture Setup (each expert's fc1 and fc2 are nn.Linear layers, which
+ * carry a bias unless told otherwise) and Full BlockFFN Layer with Combined Losses
+ * (the expert sum plus the layer's input goes through nn.LayerNorm(hidden_dim)).
+ *
+ *   b_in  [E, d_e] fp32 or NULL    fc1 biases:  h = Swish(W_in_e x + b_in_e)
+ *   b_out [E, d_h] fp32 or NULL    fc2 biases:  o_e = W_out_e h' + b_out_e; the gate
+ *                                  multiplies the whole o_e, so a token adds
+ *                                  g[t,e] b_out_e only for experts it activates
+ *   ln_weight [d_h] fp32 or NULL   when given, y = LayerNorm(sum + x): population
+ *                                  variance over d_h, scale ln_weight, shift ln_bias
+ *   ln_bias   [d_h] fp32 or NULL   (NULL: no shift; ignored without ln_weight)
+ *   ln_eps    finite, >= 0         (nn.LayerNorm's default is 1e-5)
+ * All pointers are device pointers, 16-byte aligned, owned by the caller.
+ */
+typedef struct blockffn_layer_opts {
+    const float* b_in;
+    const float* b_out;
+    const float* ln_weight;
+    const float* ln_bias;
+    float ln_eps;
+} blockffn_layer_opts;
+
+/* Flags of blockffn_forward_workspace_bytes. */
+#define BLOCKFFN_WS_ROUTER 1      /* the gates will come from the router           */
+#define BLOCKFFN_WS_EXPERT_BIAS 2 /* the calls will pass fc2 biases (opts->b_out)  */
+
+/*
  * blockffn_forward_workspace_bytes -- size of the scratch buffer blockffn_forward
- * needs for these shapes (0 when the shapes are invalid).  with_router != 0 when
- * the gates will come from the router (the workspace then also holds them).
+ * needs for these shapes (0 when the shapes are invalid).  flags: an OR of
+ * BLOCKFFN_WS_ROUTER (the gates come from the router; the workspace then also
+ * holds them) and BLOCKFFN_WS_EXPERT_BIAS (fc2 biases are given; the multi-chunk
+ * kernels then stage the per-token bias sums, T * d_h fp32, in the workspace).
+ * The value 1 means BLOCKFFN_WS_ROUTER, as the flag argument always has.
  */
 size_t blockffn_forward_workspace_bytes(int T, int d_h, int E, int d_e, int n,
-                                        blockffn_dtype dt, int with_router);
+                                        blockffn_dtype dt, int flags);
 
 /*
  * blockffn_workspace_reset -- zero a workspace (asynchronous memset on stream).
@@ -161,19 +197,28 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  * against the masks on the device, and a mismatch records
  * BLOCKFFN_ERR_INVALID_ARG in the status word (detail 11) and computes nothing.
  * W_in [E, d_e, d_h] and W_out [E, d_h, d_e] in dtype dt; y [T, d_h] in dtype dt is
- * fully overwritten (rows of tokens with no active expert are exact zeros).
+ * fully overwritten (without LayerNorm, rows of tokens with no active expert are
+ * exact zeros).  opts: NULL, or the optional biases and LayerNorm
+ * (blockffn_layer_opts); fc2 biases need a workspace sized with
+ * BLOCKFFN_WS_EXPERT_BIAS.  The single-chunk kernel applies the LayerNorm in its
+ * last step when every row tile of y has a cluster of its own (d_h <= 128 *
+ * clusters); otherwise, and on the other paths, a LayerNorm kernel follows the
+ * forward on the stream and rewrites y in place.
  * workspace: ws_bytes >= blockffn_forward_workspace_bytes(...), reset once with
  * blockffn_workspace_reset; it carries state between calls (never share one
  * workspace between calls that may overlap on the GPU).  The first call after a
- * reset binds the workspace to its (T, d_h, E, d_e, n, dt, gating mode); a later
- * call with any of these different records BLOCKFFN_ERR_WORKSPACE in the status
- * word (blockffn_get_device_status, detail 10) and computes nothing.  Reset the
- * workspace, or use another one, to change them.
+ * reset binds the workspace to its (T, d_h, E, d_e, n, dt, gating mode, whether
+ * fc2 biases are given); a later call with any of these different records
+ * BLOCKFFN_ERR_WORKSPACE in the status word (blockffn_get_device_status, detail
+ * 10) and computes nothing.  Reset the workspace, or use another one, to change
+ * them.
  * Requirements: T >= 0, 1 <= n <= 32, 1 <= E <= 256;
  *   bf16: d_h % 128 == 0, d_e % 128 == 0, d_e <= 512, E % 16 == 0 when routed;
  *   fp32: any d_h, d_e >= 1.
  * Arithmetic: bf16 inputs, fp32 accumulation; the gated Swish activations are
- * rounded to bf16 between the two GEMMs; y is rounded once to dt.
+ * rounded to bf16 between the two GEMMs; the biases and the LayerNorm are fp32;
+ * y is rounded once to dt (a LayerNorm on the single-chunk kernel works on the
+ * fp32 sum; a following LayerNorm kernel reads y as stored).
  * Kernels: one chunk (T <= n, bf16, d_h % 256 == 0) runs the single-chunk
  * cluster kernel; several chunks run the group kernel, which takes whole chunks
  * 256 tokens at a time (128 when T <= 128) and runs each expert of the group's
@@ -189,7 +234,8 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
                                  const float* b_r, const float* gamma, float eps,
                                  const int32_t* counts, const int32_t* idx, const uint32_t* tmask,
                                  const void* W_in, const void* W_out, int T, int d_h,
-                                 int E, int d_e, int n, blockffn_dtype dt, void* y,
+                                 int E, int d_e, int n, blockffn_dtype dt,
+                                 const blockffn_layer_opts* opts, void* y,
                                  void* workspace, size_t ws_bytes, void* stream);
 
 /*

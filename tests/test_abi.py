@@ -74,7 +74,7 @@ def test_forward_rejects_bad_shapes_on_host(lib, T, d_h, E, d_e, n, dt):
     L = lib.lib
     assert L.blockffn_forward_workspace_bytes(T, d_h, E, d_e, n, dt, 0) == 0
     st = L.blockffn_forward(16, 16, None, None, None, 0.0, None, None, None, 16, 16, T, d_h, E, d_e,
-                            n, dt, 16, 16, 1 << 30, None)
+                            n, dt, None, 16, 16, 1 << 30, None)
     assert st in (lib.ERR_INVALID_ARG, lib.ERR_UNSUPPORTED)
     assert L.blockffn_last_error_message()
 
@@ -84,11 +84,11 @@ def test_forward_gating_source_is_exclusive(lib):
     # (T = 32 > 0: with T = 0 the call is a no-op before this check)
     # gates and router weights together
     st = L.blockffn_forward(16, 16, 16, None, None, 0.0, None, None, None, 16, 16, 32, 2048, 64, 128,
-                            32, 1, 16, 16, 1 << 30, None)
+                            32, 1, None, 16, 16, 1 << 30, None)
     assert st == lib.ERR_INVALID_ARG
     # neither
     st = L.blockffn_forward(16, None, None, None, None, 0.0, None, None, None, 16, 16, 32, 2048, 64,
-                            128, 32, 1, 16, 16, 1 << 30, None)
+                            128, 32, 1, None, 16, 16, 1 << 30, None)
     assert st == lib.ERR_INVALID_ARG
 
 
@@ -96,7 +96,7 @@ def test_forward_union_tables_all_or_none(lib):
     """counts, idx and tmask come together or not at all, only with injected gates,
     and 16-byte aligned; each refusal is made on the host."""
     L = lib.lib
-    args = (16, 16, 32, 2048, 64, 128, 32, 1, 16, 16, 1 << 30, None)
+    args = (16, 16, 32, 2048, 64, 128, 32, 1, None, 16, 16, 1 << 30, None)
     # two of the three
     assert L.blockffn_forward(16, 16, None, None, None, 0.0, 16, 16, None, *args) == lib.ERR_INVALID_ARG
     assert L.blockffn_forward(16, 16, None, None, None, 0.0, None, None, 16, *args) == lib.ERR_INVALID_ARG
@@ -105,6 +105,28 @@ def test_forward_union_tables_all_or_none(lib):
     assert b"injected" in L.blockffn_last_error_message()
     # misaligned table
     assert L.blockffn_forward(16, 16, None, None, None, 0.0, 16, 20, 16, *args) == lib.ERR_INVALID_ARG
+
+
+def test_forward_layer_options_checked_on_host(lib):
+    """Expert biases and the LayerNorm (blockffn_layer_opts): misaligned pointers and
+    a bad ln_eps are refused on the host; unknown workspace flags size nothing."""
+    import ctypes
+    L = lib.lib
+    args = (16, 16, 32, 2048, 64, 128, 32, 1)
+    tail = (16, 16, 1 << 30, None)
+
+    def call(opts):
+        return L.blockffn_forward(16, 16, None, None, None, 0.0, None, None, None, *args,
+                                  ctypes.byref(opts), *tail)
+
+    assert call(lib.LayerOpts(20, None, None, None, 0.0)) == lib.ERR_INVALID_ARG        # b_in
+    assert call(lib.LayerOpts(None, 24, None, None, 0.0)) == lib.ERR_INVALID_ARG        # b_out
+    assert call(lib.LayerOpts(None, None, 20, None, 1e-5)) == lib.ERR_INVALID_ARG       # ln_weight
+    assert call(lib.LayerOpts(None, None, 16, 20, 1e-5)) == lib.ERR_INVALID_ARG         # ln_bias
+    assert call(lib.LayerOpts(None, None, 16, None, -1.0)) == lib.ERR_INVALID_ARG       # ln_eps < 0
+    assert call(lib.LayerOpts(None, None, 16, None, float("inf"))) == lib.ERR_INVALID_ARG
+    assert b"ln_eps" in L.blockffn_last_error_message()
+    assert L.blockffn_forward_workspace_bytes(32, 2048, 64, 128, 32, 1, 4) == 0          # unknown flag
 
 
 def test_union_and_route_reject_bad_args(lib):
@@ -127,7 +149,7 @@ def test_residual_layernorm_rejects_bad_args(lib):
     assert f(16, 16, 16, 16, -1.0, 4, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG   # eps < 0
     assert f(16, 16, 16, 16, float("nan"), 4, 64, lib.F32, 16, None) == lib.ERR_INVALID_ARG
     assert f(None, 16, 16, 16, 1e-5, 4, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG  # null y
-    assert f(16, 16, 16, None, 1e-5, 4, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG  # null shift
+    assert f(16, 16, None, 16, 1e-5, 4, 64, lib.BF16, 16, None) == lib.ERR_INVALID_ARG  # null scale
     # no rows: nothing to do, nothing launched, no pointer needed
     assert f(None, None, None, None, 1e-5, 0, 64, lib.BF16, None, None) == lib.OK
 
@@ -138,4 +160,4 @@ def test_empty_inputs_are_no_ops(lib):
     assert L.blockffn_chunk_union(None, 0, 64, 32, None, None, None, None) == lib.OK
     assert L.blockffn_route(None, None, None, None, 0.0, 0, 64, 16, 1, None, None) == lib.OK
     assert L.blockffn_forward(None, 16, None, None, None, 0.0, None, None, None, None, None, 0, 2048,
-                              64, 128, 32, 1, None, None, 0, None) == lib.OK
+                              64, 128, 32, 1, None, None, None, 0, None) == lib.OK

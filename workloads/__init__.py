@@ -142,6 +142,25 @@ def expert_weights(seed: int, E: int, d_e: int, d_h: int, dtype: str):
     return W_in, W_out
 
 
+def _uniform(seed: int, stream: int, shape, bound: float) -> np.ndarray:
+    return _rng(seed, stream).uniform(-bound, bound, shape)
+
+
+def expert_biases(seed: int, E: int, d_e: int, d_h: int, scale: float = 1.0):
+    """fc1 biases [E, d_e] and fc2 biases [E, d_h], fp32: nn.Linear's initial
+    distribution U(-1/sqrt(fan_in), 1/sqrt(fan_in)) times ``scale``."""
+    b_in = _uniform(seed, 7, (E, d_e), scale / np.sqrt(d_h)).astype(np.float32)
+    b_out = _uniform(seed, 8, (E, d_h), scale / np.sqrt(d_e)).astype(np.float32)
+    return b_in, b_out
+
+
+def layernorm_params(seed: int, d_h: int):
+    """LayerNorm scale U(0.5, 1.5) and shift N(0, 0.1^2), fp32 [d_h] each."""
+    w = _rng(seed, 9).uniform(0.5, 1.5, d_h).astype(np.float32)
+    b = (0.1 * _rng(seed, 10).standard_normal(d_h)).astype(np.float32)
+    return w, b
+
+
 def router_weights(seed: int, E: int, d_h: int, dtype: str):
     return _round(normal(seed, 2, (E, d_h), 1.0 / np.sqrt(d_h)), dtype)
 
