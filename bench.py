@@ -692,6 +692,40 @@ def main():
     routed_us = graph_us(lambda i: bffn.forward(bufs[i]["x"], bufs[i]["W_in"], bufs[i]["W_out"], n, W_r=W_r[i],
                                                 gamma=gam, eps=2.0 ** -23, y=bufs[i]["y"], workspace=ws_r))
 
+    # the layer's optional parts, context only: the same decode step with the
+    # experts' fc1/fc2 biases and with LayerNorm(y + x) in the kernel's last step,
+    # beside the plain step followed by the LayerNorm kernel
+    bi_np, bo_np = wl.expert_biases(7, E, d_e, d_h)
+    lw_np, lb_np = wl.layernorm_params(7, d_h)
+    f32d = lambda a: torch.from_numpy(a).to(device=dev, dtype=torch.float32)
+    b_in_t, b_out_t, lw_t, lb_t = f32d(bi_np), f32d(bo_np), f32d(lw_np), f32d(lb_np)
+    ws_o = bffn.Workspace.for_shapes(T, d_h, E, d_e, n, dt, False, dev, with_bias=True)
+
+    def opt_step(i, biases=False, ln=False):
+        b = bufs[i]
+        bffn.forward(b["x"], b["W_in"], b["W_out"], n, gates=b["g"], y=b["y"], workspace=ws_o,
+                     b_in=b_in_t if biases else None, b_out=b_out_t if biases else None,
+                     ln_weight=lw_t if ln else None, ln_bias=lb_t if ln else None)
+
+    def plain_then_ln(i):
+        b = bufs[i]
+        bffn.forward(b["x"], b["W_in"], b["W_out"], n, gates=b["g"], y=b["y"], workspace=ws)
+        bffn.residual_layernorm(b["y"], b["x"], lw_t, lb_t, 1e-5, out=b["y"])
+
+    layer_opts = {
+        "plain_step_us": graph_us(lambda i: opt_step(i)),
+        "biases_step_us": graph_us(lambda i: opt_step(i, biases=True)),
+        "layernorm_in_kernel_step_us": graph_us(lambda i: opt_step(i, ln=True)),
+        "biases_and_layernorm_step_us": graph_us(lambda i: opt_step(i, biases=True, ln=True)),
+        "step_then_layernorm_kernel_us": graph_us(plain_then_ln),
+        "what": "chunk32 decode step with fc1/fc2 biases (nn.Linear init) and/or LayerNorm(y + x) applied "
+                "in the single-chunk kernel's last step; against the plain step followed by the "
+                "LayerNorm kernel; CUDA-graph replays over the rotating copies",
+    }
+    st_o = bffn.device_status(ws_o)
+    if st_o[0] != 0:
+        raise SystemExit(f"device status {st_o} after the layer-option steps")
+
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline()
@@ -742,6 +776,7 @@ def main():
                            "step; a CUDA graph of 8 steps (copies on two side streams, overlapping the "
                            "neighbouring steps' kernels), replayed"},
             "gpu_launches": args.steps,
+            "layer_options": layer_opts,
             "routed_decode": {"router_us": router_us, "step_us": routed_us,
                               "what": "router (tensor cores) + single-chunk forward, gates from a seeded "
                                       "router instead of injected; graph replay"},

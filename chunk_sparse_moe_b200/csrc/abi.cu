@@ -141,7 +141,7 @@ struct Layout {
     size_t ctl, counts, offsets, idx, tmask, pair_ce, gcounts, goffsets, gpair, gates;
     size_t readyA, cntB, partB, hbuf;
     size_t ybias;        // group path with fc2 biases: [T, d_h] fp32 per-token bias sums
-    size_t lnstats;      // single-chunk path: [RT*4][32] (mean, M2) of the LayerNorm slices
+    size_t lnstats;      // single-chunk path: [32][RT*4] (mean, M2) of the LayerNorm slices
     size_t total;
     int C;               // chunks
     int N;               // tokens per MMA
@@ -225,6 +225,7 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         L.cntB = take(2 * NGr * L.RT * 4);
         L.partB = take((size_t)G * 2 * L.N * 128 * 4);
         L.hbuf = take(Pm * L.N * d_e * 2);
+        // last, so that every other offset is the same with or without it
         if (with_bias) L.ybias = take((size_t)T * d_h * 4);
     }
     L.total = off;
@@ -469,7 +470,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.skip_unit = g_skip_flag.load();
         da.wait_ns = g_wait_ns.load();
         da.trace = g_trace.load();
-        da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1, Gd, with_bias ? 1 : 0});
+        da.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 1, Gd});
         // A cluster launch cannot also be cooperative; the grid is sized to the
         // clusters that can be resident at once, and every wait is bounded.
         e = launch_forward_decode(da, dmaps, Gd, s);
@@ -529,7 +530,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     a.KBe = L.KBe;
     a.skip_flag_unit = g_skip_flag.load();
     a.wait_ns = g_wait_ns.load();
-    a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2, G, with_bias ? 1 : 0});
+    a.shape_key = shape_key({T, d_h, E, d_e, n, (long long)dt, routed ? 1 : 0, 2, G});
     a.trace = g_trace.load();
     e = launch_forward_group(a, maps, G, s);
     if (e != cudaSuccess) return cuda_fail(e, "group forward launch");

@@ -641,7 +641,7 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             named_bar_sync(1, kGrEpi);
             if (et == 0) {
                 GR_TRACE(kGtAnnounce);
-                __threadfence();
+                fence_acq_rel_gpu();
                 for (long long u = uLo; u < uHi; ++u)
                     if ((int)u != a.skip_flag_unit) atomicAdd(&readyA[u], 1u);
                 mbar_arrive(&sh.a_pub);
@@ -653,7 +653,7 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             named_bar_sync(1, kGrEpi);
             if (et == 0) {
                 GR_TRACE(kGtLoopEnd);
-                __threadfence();
+                fence_acq_rel_gpu();
                 if (npend >= 1) atomicAdd(cntB + pend_sg[0].unit, 1u);
                 if (npend >= 2) atomicAdd(cntB + pend_sg[1].unit, 1u);
                 GR_TRACE(kGtFlushAnnounced);

@@ -108,7 +108,7 @@ struct DcArgs {
     const float* ln_w;
     const float* ln_b;
     float ln_eps;
-    float2* ln_stats;         // [RT*4 slices][32 tokens] (mean, M2) of a 32-row slice
+    float2* ln_stats;         // [32 tokens][RT*4 slices] (mean, M2) of a 32-row slice
     int T, d_h, E, d_e, n, N;
     int KB;    // d_h / 64
     int RT;    // d_h / 128

@@ -226,12 +226,12 @@ __global__ void __launch_bounds__(kGpThreads) group_union_plan_kernel(
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();   // this block's tables before its count
+        fence_acq_rel_gpu();   // this block's tables before its count
         s_last = atomicAdd(&ctl->plan_done, 1u) == gridDim.x - 1;
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();       // every block's tables after the count that saw them all
+    fence_acq_rel_gpu();       // every block's tables after the count that saw them all
     if (threadIdx.x == 0) ctl->plan_done = 0u;
     if (plan_refused(ctl)) return;   // refused tables or an earlier error: compute nothing
     for (int g = warp; g < NGr; g += nwarps) {

@@ -9,10 +9,11 @@ Deployment", Full BlockFFN Layer with Combined Losses (a layer is the expert
 sum, then the residual and LayerNorm).
 
 A verification step takes the hidden states of n drafted tokens and runs every
-layer on them: ``forward`` (the union of the chunk's experts, gates either
-injected per layer or from the layer's router) and ``residual_layernorm``, all
-issued on one stream with no host synchronisation (each kernel is a
-programmatic dependent of the one before it).  There is no draft model and no
+layer on them: one ``forward`` per layer (the union of the chunk's experts,
+gates either injected per layer or from the layer's router, optional expert
+biases, and the closing LayerNorm(y + h), which the single-chunk kernel applies
+in its last step), all issued on one stream with no host synchronisation (each
+kernel is a programmatic dependent of the one before it).  There is no draft model and no
 language-model head: how many tokens a step accepts is a synthetic input (see
 ``workloads.accept_lengths``), so the driver measures the verifier's cost per
 drafted and per accepted token.  Only orchestration lives here; every step of
@@ -25,7 +26,7 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from .api import Workspace, forward, residual_layernorm
+from .api import Workspace, forward
 
 
 @dataclass
@@ -40,6 +41,8 @@ class Layer:
     gamma: Optional[torch.Tensor] = None     # [E] fp32
     eps: float = 2.0 ** -23                  # router RMSNorm epsilon
     ln_eps: float = 1e-5                     # LayerNorm epsilon
+    b_in: Optional[torch.Tensor] = None      # [E, d_e] fp32 expert fc1 biases
+    b_out: Optional[torch.Tensor] = None     # [E, d_h] fp32 expert fc2 biases
 
 
 class Verifier:
@@ -57,8 +60,8 @@ class Verifier:
         self.d_h = d_h
         device = device or self.layers[0].W_in.device
         self.ws = [Workspace.for_shapes(n, L.W_in.shape[2], L.W_in.shape[0], L.W_in.shape[1], n, dtype,
-                                        L.gates is None, device) for L in self.layers]
-        self.y = torch.empty((n, d_h), dtype=dtype, device=device)
+                                        L.gates is None, device, with_bias=L.b_out is not None)
+                   for L in self.layers]
         self.h = [torch.empty((n, d_h), dtype=dtype, device=device) for _ in range(2)]
 
     def step(self, x: torch.Tensor) -> torch.Tensor:
@@ -66,12 +69,13 @@ class Verifier:
         verifier's, overwritten by the next step)."""
         h = x
         for i, L in enumerate(self.layers):
+            # the layer's output goes to the buffer its input is not in
+            kw = dict(y=self.h[i % 2], workspace=self.ws[i], b_in=L.b_in, b_out=L.b_out,
+                      ln_weight=L.ln_gamma, ln_bias=L.ln_beta, ln_eps=L.ln_eps)
             if L.gates is not None:
-                y = forward(h, L.W_in, L.W_out, self.n, gates=L.gates, y=self.y, workspace=self.ws[i])
+                h = forward(h, L.W_in, L.W_out, self.n, gates=L.gates, **kw)
             else:
-                y = forward(h, L.W_in, L.W_out, self.n, W_r=L.W_r, b_r=L.b_r, gamma=L.gamma, eps=L.eps,
-                            y=self.y, workspace=self.ws[i])
-            h = residual_layernorm(y, h, L.ln_gamma, L.ln_beta, L.ln_eps, out=self.h[i % 2])
+                h = forward(h, L.W_in, L.W_out, self.n, W_r=L.W_r, b_r=L.b_r, gamma=L.gamma, eps=L.eps, **kw)
         return h
 
 

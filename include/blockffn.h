@@ -207,11 +207,11 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  * workspace: ws_bytes >= blockffn_forward_workspace_bytes(...), reset once with
  * blockffn_workspace_reset; it carries state between calls (never share one
  * workspace between calls that may overlap on the GPU).  The first call after a
- * reset binds the workspace to its (T, d_h, E, d_e, n, dt, gating mode, whether
- * fc2 biases are given); a later call with any of these different records
- * BLOCKFFN_ERR_WORKSPACE in the status word (blockffn_get_device_status, detail
- * 10) and computes nothing.  Reset the workspace, or use another one, to change
- * them.
+ * reset binds the workspace to its (T, d_h, E, d_e, n, dt, gating mode); a later
+ * call with any of these different records BLOCKFFN_ERR_WORKSPACE in the status
+ * word (blockffn_get_device_status, detail 10) and computes nothing.  Reset the
+ * workspace, or use another one, to change them.  Calls with and without the
+ * optional parts may share a workspace (one sized for fc2 biases serves both).
  * Requirements: T >= 0, 1 <= n <= 32, 1 <= E <= 256;
  *   bf16: d_h % 128 == 0, d_e % 128 == 0, d_e <= 512, E % 16 == 0 when routed;
  *   fp32: any d_h, d_e >= 1.

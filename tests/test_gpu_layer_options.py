@@ -129,18 +129,20 @@ def test_options_deterministic(bffn):
     assert np.array_equal(y1, y2)
 
 
-def test_layernorm_alternating_with_plain_calls(bffn):
-    """One workspace, calls with and without the fused LayerNorm in turn: the
-    per-launch slice counters stay in step."""
-    w = wl.chunk32(seed=6)
+@pytest.mark.parametrize("T", [32, 300])
+def test_options_alternating_on_one_workspace(bffn, T):
+    """One workspace (sized for fc2 biases), calls with and without biases and the
+    LayerNorm in turn: the layout and the per-launch counters stay in step."""
+    w = wl.make_injected("alt", T, 32, 2048 if T == 32 else 512, 64, 128, "bf16", "markov80", seed=6)
     ws = bffn.Workspace.for_shapes(w.T, w.d_h, w.E, w.d_e, w.n, torch.bfloat16, False, "cuda",
                                    with_bias=True)
     p = _params(w, 6)
-    for k in range(5):
-        use_ln = k % 2 == 0
-        y, g = _run(bffn, w, p[0], p[1], p[2] if use_ln else None, p[3] if use_ln else None, workspace=ws)
-        assert_close(y, _ref(w, g, p[0], p[1], p[2] if use_ln else None, p[3] if use_ln else None), "bf16",
-                     f"call {k}")
+    for k in range(6):
+        use_ln, use_b = k % 2 == 0, k % 3 != 2
+        q = (p[0] if use_b else None, p[1] if use_b else None, p[2] if use_ln else None,
+             p[3] if use_ln else None)
+        y, g = _run(bffn, w, *q, workspace=ws)
+        assert_close(y, _ref(w, g, *q), "bf16", f"call {k}")
     assert bffn.device_status(ws) == (0, 0)
 
 

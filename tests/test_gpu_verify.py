@@ -1,10 +1,11 @@
 """GPU: the synthetic speculative-verification driver (a stack of layers over
-one draft chunk: forward, then residual + LayerNorm, chained on one stream).
+one draft chunk: each layer one forward with expert biases and the closing
+residual + LayerNorm, chained on one stream).
 
 The oracle chain mirrors the dataflow: every layer consumes the previous
-layer's output as stored (bf16), y is rounded to bf16 before the LayerNorm and
-the LayerNorm's output to bf16, each step in fp64 (oracle.forward_chunk_union,
-oracle.residual_layernorm).
+layer's output as stored (bf16); within a layer the expert sum stays unrounded
+into the LayerNorm, whose output is rounded to bf16, each step in fp64
+(oracle.forward_chunk_union with the biases, oracle.residual_layernorm).
 """
 import numpy as np
 import pytest
@@ -25,9 +26,12 @@ def bffn():
 def _stack(bffn, L, n, d_h, E, d_e, seed=0):
     from chunk_sparse_moe_b200.verify import Layer
     raw = wl.layer_stack(L, n, d_h, E, d_e, "bf16", seed=seed)
+    for i, r in enumerate(raw):
+        r["b_in"], r["b_out"] = wl.expert_biases(seed * 100 + i, E, d_e, d_h)
     layers = [Layer(W_in=dev(r["W_in"], torch.bfloat16), W_out=dev(r["W_out"], torch.bfloat16),
                     ln_gamma=dev(r["ln_gamma"], torch.float32), ln_beta=dev(r["ln_beta"], torch.float32),
-                    gates=dev(r["gates"], torch.float32)) for r in raw]
+                    gates=dev(r["gates"], torch.float32), b_in=dev(r["b_in"], torch.float32),
+                    b_out=dev(r["b_out"], torch.float32)) for r in raw]
     return raw, layers
 
 
@@ -40,7 +44,7 @@ def test_layer_stack_matches_the_oracle_chain(bffn):
     h = to_np64(v.step(dev(x, torch.bfloat16)))
     ref = x.astype(np.float64)
     for r in raw:
-        y = wl.bf16_round(oracle.forward_chunk_union(ref, r["gates"], r["W_in"], r["W_out"], n))
+        y = oracle.forward_chunk_union(ref, r["gates"], r["W_in"], r["W_out"], n, r["b_in"], r["b_out"])
         ref = wl.bf16_round(oracle.residual_layernorm(y, ref, r["ln_gamma"], r["ln_beta"], 1e-5))
     assert_close(h, ref.astype(np.float64), "bf16", "3-layer chain")
 
@@ -59,9 +63,8 @@ def test_chained_steps_equal_synchronised_layers(bffn):
     torch.cuda.synchronize()
     h = x
     for i, L in enumerate(layers):
-        y = bffn.forward(h, L.W_in, L.W_out, n, gates=L.gates, workspace=v.ws[i])
-        torch.cuda.synchronize()
-        h = bffn.residual_layernorm(y, h, L.ln_gamma, L.ln_beta, 1e-5)
+        h = bffn.forward(h, L.W_in, L.W_out, n, gates=L.gates, workspace=v.ws[i], b_in=L.b_in, b_out=L.b_out,
+                         ln_weight=L.ln_gamma, ln_bias=L.ln_beta, ln_eps=1e-5)
         torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert torch.equal(a, h)
