@@ -693,8 +693,7 @@ def main():
                                                 gamma=gam, eps=2.0 ** -23, y=bufs[i]["y"], workspace=ws_r))
 
     # the layer's optional parts, context only: the same decode step with the
-    # experts' fc1/fc2 biases and with LayerNorm(y + x) in the kernel's last step,
-    # beside the plain step followed by the LayerNorm kernel
+    # experts' fc1/fc2 biases and with LayerNorm(y + x)
     bi_np, bo_np = wl.expert_biases(7, E, d_e, d_h)
     lw_np, lb_np = wl.layernorm_params(7, d_h)
     f32d = lambda a: torch.from_numpy(a).to(device=dev, dtype=torch.float32)
@@ -715,12 +714,13 @@ def main():
     layer_opts = {
         "plain_step_us": graph_us(lambda i: opt_step(i)),
         "biases_step_us": graph_us(lambda i: opt_step(i, biases=True)),
-        "layernorm_in_kernel_step_us": graph_us(lambda i: opt_step(i, ln=True)),
+        "layernorm_step_us": graph_us(lambda i: opt_step(i, ln=True)),
         "biases_and_layernorm_step_us": graph_us(lambda i: opt_step(i, biases=True, ln=True)),
-        "step_then_layernorm_kernel_us": graph_us(plain_then_ln),
-        "what": "chunk32 decode step with fc1/fc2 biases (nn.Linear init) and/or LayerNorm(y + x) applied "
-                "in the single-chunk kernel's last step; against the plain step followed by the "
-                "LayerNorm kernel; CUDA-graph replays over the rotating copies",
+        "step_then_layernorm_call_us": graph_us(plain_then_ln),
+        "what": "chunk32 decode step through blockffn_forward with fc1/fc2 biases (nn.Linear init) and/or "
+                "LayerNorm(y + x) (the LayerNorm kernel follows the forward as its programmatic "
+                "dependent); beside it the plain step and a separate blockffn_residual_layernorm call; "
+                "CUDA-graph replays over the rotating copies",
     }
     st_o = bffn.device_status(ws_o)
     if st_o[0] != 0:

@@ -141,7 +141,6 @@ struct Layout {
     size_t ctl, counts, offsets, idx, tmask, pair_ce, gcounts, goffsets, gpair, gates;
     size_t readyA, cntB, partB, hbuf;
     size_t ybias;        // group path with fc2 biases: [T, d_h] fp32 per-token bias sums
-    size_t lnstats;      // single-chunk path: [32][RT*4] (mean, M2) of the LayerNorm slices
     size_t total;
     int C;               // chunks
     int N;               // tokens per MMA
@@ -186,7 +185,7 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         return o;
     };
     L.ctl = L.counts = L.offsets = L.idx = L.tmask = L.pair_ce = L.gcounts = L.goffsets = L.gpair = 0;
-    L.gates = L.readyA = L.cntB = L.partB = L.hbuf = L.ybias = L.lnstats = 0;
+    L.gates = L.readyA = L.cntB = L.partB = L.hbuf = L.ybias = 0;
     L.NG = L.NT = L.NGr = 0;
     const size_t C = (size_t)L.C;
     L.ctl = take(sizeof(Ctl));
@@ -206,7 +205,6 @@ void make_layout(int T, int d_h, int E, int d_e, int n, bool bf16, bool with_rou
         L.Pmax = E;
         L.readyA = take(2 * (size_t)E * 4);
         L.hbuf = take((size_t)E * L.N * d_e * 2);
-        L.lnstats = take((size_t)L.RT * 4 * 32 * 8);
     } else {
         // groups of whole chunks, N = 128 tokens per MMA for short inputs, else 256
         L.N = T <= 128 ? 128 : 256;
@@ -390,7 +388,8 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
     if (ws_bytes < L.total)
         return fail(BLOCKFFN_ERR_WORKSPACE, "workspace of %zu bytes < %zu needed%s", ws_bytes, L.total,
                     with_bias ? " (fc2 biases: size it with BLOCKFFN_WS_EXPERT_BIAS)" : "");
-    // the LayerNorm as its own kernel after the forward, rewriting y in place
+    // the LayerNorm as its own kernel after the forward (a programmatic dependent
+    // of it), rewriting y in place
     auto closing_layernorm = [&]() -> blockffn_status {
         if (!ln_w) return BLOCKFFN_OK;
         cudaError_t e2 = launch_residual_layernorm(y, x, ln_w, ln_b, ln_eps, T, d_h, bf16, y,
@@ -449,16 +448,8 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         da.hbuf = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
         da.readyA = reinterpret_cast<uint32_t*>(ws + L.readyA);
         da.ctl = ctl;
-        da.x = static_cast<const __nv_bfloat16*>(x);
         da.b_in = b_in;
         da.b_out = b_out;
-        // the LayerNorm in the kernel's last step when every row tile of y has a
-        // cluster of its own, else as a kernel of its own afterwards
-        const bool ln_fused = ln_w != nullptr && L.RT <= Gd / 4;
-        da.ln_w = ln_fused ? ln_w : nullptr;
-        da.ln_b = ln_fused ? ln_b : nullptr;
-        da.ln_eps = ln_eps;
-        da.ln_stats = reinterpret_cast<float2*>(ws + L.lnstats);
         da.T = T;
         da.d_h = d_h;
         da.E = E;
@@ -475,7 +466,7 @@ blockffn_status blockffn_forward(const void* x, const float* gates, const void* 
         // clusters that can be resident at once, and every wait is bounded.
         e = launch_forward_decode(da, dmaps, Gd, s);
         if (e != cudaSuccess) return cuda_fail(e, "single-chunk forward launch");
-        return ln_fused ? BLOCKFFN_OK : closing_layernorm();
+        return closing_layernorm();
     }
 
     // several chunks (or one the single-chunk kernel cannot take): group tables,
@@ -621,13 +612,8 @@ blockffn_status blockffn_forward_noalloc(const void* x, const float* gates, cons
     da.hbuf = reinterpret_cast<__nv_bfloat16*>(scratch + off_h);
     da.readyA = reinterpret_cast<uint32_t*>(scratch + off_ready);
     da.ctl = reinterpret_cast<Ctl*>(scratch);
-    da.x = static_cast<const __nv_bfloat16*>(x);
     da.b_in = nullptr;
     da.b_out = nullptr;
-    da.ln_w = nullptr;
-    da.ln_b = nullptr;
-    da.ln_eps = 0.f;
-    da.ln_stats = nullptr;
     da.T = T;
     da.d_h = d_h;
     da.E = E;

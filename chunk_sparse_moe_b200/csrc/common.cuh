@@ -52,10 +52,7 @@ struct Ctl {
     // a workspace by its shape key), so ticket / G is the launch's index with one
     // atomic and no end-of-launch bookkeeping.  64 bits: it never wraps.
     unsigned long long ticket;
-    // by launch parity: 32-row slices of y whose LayerNorm statistics the
-    // single-chunk kernel has published (each launch zeroes the next one's word)
-    uint32_t ln_cnt[2];
-    uint32_t pad[52];
+    uint32_t pad[54];
 };
 static_assert(sizeof(Ctl) == 256, "control block is 256 bytes");
 

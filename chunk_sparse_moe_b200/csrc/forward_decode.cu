@@ -33,21 +33,14 @@
 // block of rank q, which adds the 4 contributions in rank order (a fixed order)
 // and writes those 32 rows of y.
 //
-// Optional parts of the layer (the experts' nn.Linear biases, Router
-// Architecture Setup; the closing LayerNorm, Full BlockFFN Layer with Combined
-// Losses).  The fc1 bias of an accumulator row is added before Swish.  The
-// summing warp of a row slice adds, before the four partials, the gated fc2
-// biases of its rows: sum over the union, ascending, of bit_t ? g[t,e] b_out[e,i]
-// : 0 (computed while the expert-out MMAs run).  With a LayerNorm, v = sum + x
-// stays in fp32: each summing warp publishes its 32-row slice's per-token mean
-// and sum of squared deviations, counts the slice in (release), waits (bounded)
-// until every slice of y is counted in, forms each token's mean and variance from
-// the slices (the two-level decomposition of the variance: exact, and in a fixed
-// order), and stores ln_w * (v - mean) / sqrt(var + eps) + ln_b.
-// The four epilogue warps then share the loads of the statistics (a quarter of
-// the slices each) and the summing warp normalises its rows from its own receive
-// slot.  That needs every row tile of y summed by a cluster of its own (one slice
-// per summing warp); the host otherwise runs the LayerNorm as a following kernel.
+// Optional expert biases (the experts' nn.Linear layers, Router Architecture
+// Setup).  The fc1 bias of an accumulator row is added before Swish.  The summing
+// warp of a row slice starts from the gated fc2 biases of its rows, sum over the
+// union, ascending, of bit_t ? g[t,e] b_out[e,i] : 0 (formed while the
+// expert-out MMAs run), and adds the four partials to it.  (The layer's closing
+// LayerNorm runs as a kernel of its own after this one: done here, its
+// statistics would need every cluster's rows before any row could be stored,
+// and that chain measured slower than the separate launch.)
 //
 // Roles (224 threads): warp 0 TMA producer (one lane), warp 1 MMA issuer (the
 // whole warp runs its loops and waits, one elected lane issues), warp 2 TMEM
@@ -112,7 +105,6 @@ struct RsShared {
     int ep_okA[2];                // epilogue: the two waits of an expert-in unit
     int ep_okB[2];                // epilogue: the two waits of an expert-out row tile
     int b_go, b_fail;             // epilogue: expert-out work may start / a summing warp gave up
-    int ln_ok;                    // epilogue: every slice's LayerNorm statistics are published
     uint32_t epoch;
     int P;
     uint32_t trace_once;          // trace slots already stamped (first occurrence only)
@@ -127,8 +119,7 @@ enum : int {
     kRtStart = 0, kRtPrologue = 1, kRtFirstLoad = 2, kRtLastLoad = 3, kRtFirstFull = 4,
     kRtLastACommit = 5, kRtADone = 7, kRtFirstFlag = 8, kRtLastFlag = 9, kRtLastCommit = 10,
     kRtLastEpi = 11, kRtEnd = 13, kRtATmem = 14, kRtASent = 15, kRtAReady = 16, kRtARead = 17,
-    kRtAWritten = 18, kRtBSent = 21, kRtBReduced = 23, kRtFirstBMma = 24, kRtLnPublished = 25,
-    kRtLnSeen = 26, kRtLnCombined = 27, kRtBRecv = 30, kRtLnEnter = 31, kRtSlots = 64
+    kRtAWritten = 18, kRtBSent = 21, kRtBReduced = 23, kRtFirstBMma = 24, kRtBRecv = 30, kRtSlots = 64
 };
 #define RS_TRACE(slot) \
     do { if (a.trace) a.trace[(size_t)blockIdx.x * kRtSlots + (slot)] = globaltimer_ns(); } while (0)
@@ -329,11 +320,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const unsigned long long tk = atomicAdd(&a.ctl->ticket, 1ull);
         const unsigned long long key0 = claim_shape_key(a.ctl, a.shape_key);
         const uint32_t ep0 = (uint32_t)(tk / gridDim.x);
-        if (blockIdx.x == 0) {
-            // the next launch's counters
-            a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;
-            a.ctl->ln_cnt[(ep0 & 1u) ^ 1u] = 0u;
-        }
+        if (blockIdx.x == 0) a.ctl->issued[(ep0 & 1u) ^ 1u] = 0u;   // the next launch's counter
         sh.epoch = ep0;
         const bool key_ok = key0 == 0ull || key0 == a.shape_key;
         if (!key_ok) record_error(a.ctl, kErrWorkspace, kShapeKey);
@@ -660,30 +647,8 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // meet the same named barriers.
         bool failed = abort_at_start;
         if (P == 0 && blockIdx.x == 0 && !failed) {
-            if (a.ln_w == nullptr) {
-                // empty union: y is all zeros
-                for (size_t k2 = et; k2 < (size_t)nt * a.d_h; k2 += 128) a.y[k2] = __float2bfloat16_rn(0.f);
-            } else {
-                // empty union: the expert sum is zero, y = LayerNorm(x); warp w
-                // takes tokens w, w + 4, ... (two passes over the row, then the store)
-                for (int t = warp - 3; t < nt; t += 4) {
-                    const __nv_bfloat16* xr = a.x + (size_t)t * a.d_h;
-                    float sm = 0.f;
-                    for (int k2 = lane; k2 < a.d_h; k2 += 32) sm += __bfloat162float(xr[k2]);
-                    const float mu = rs_warp_allsum(sm) / (float)a.d_h;
-                    float q = 0.f;
-                    for (int k2 = lane; k2 < a.d_h; k2 += 32) {
-                        const float dv = __bfloat162float(xr[k2]) - mu;
-                        q = fmaf(dv, dv, q);
-                    }
-                    const float rstd = 1.0f / sqrtf(rs_warp_allsum(q) / (float)a.d_h + a.ln_eps);
-                    for (int k2 = lane; k2 < a.d_h; k2 += 32) {
-                        const float o = a.ln_w[k2] * ((__bfloat162float(xr[k2]) - mu) * rstd) +
-                                        (a.ln_b != nullptr ? a.ln_b[k2] : 0.f);
-                        a.y[(size_t)t * a.d_h + k2] = __float2bfloat16_rn(o);
-                    }
-                }
-            }
+            // empty union: y is all zeros
+            for (size_t k2 = et; k2 < (size_t)nt * a.d_h; k2 += 128) a.y[k2] = __float2bfloat16_rn(0.f);
         }
         // ---- A units: each block finishes its half of the tokens
         const uint32_t peer = (uint32_t)(wk.cr ^ 1);
@@ -851,15 +816,6 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                                 bacc[t] = fmaf(__shfl_sync(0xffffffffu, gl[u], t), bv[u], bacc[t]);
                     }
                 }
-                // with the LayerNorm, the residual x of this warp's rows joins the bias
-                // sums here (loaded before the waits below): the summing warp then
-                // forms v = x + biases + the four partials
-                if (a.ln_w != nullptr && qd == wk.cr) {
-                    const __nv_bfloat16* xr = a.x + rt * 128 + wk.cr * 32 + lane;
-#pragma unroll
-                    for (int t = 0; t < N; ++t)
-                        if (t < nt) bacc[t] += __bfloat162float(xr[(size_t)t * a.d_h]);
-                }
                 if (nBt > 0) {
                     if (et == 0)
                         sh.ep_okB[0] = wait_bar(&sh.accB_full[ab], (uint32_t)((k >> 1) & 1), limit, &sh.abort, a.ctl,
@@ -932,44 +888,8 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                                 }
                             }
                         }
-                        if (a.ln_w != nullptr) {
-                            // LayerNorm(sum + x), first half: v (x included) goes to this
-                            // rank's own receive slot (no peer writes there), [N tokens]
-                            // [32 rows]; lane t forms token t's mean and M2 over the
-                            // slice's 32 rows (a rotated walk: no bank conflicts) and
-                            // publishes them; the four epilogue warps finish after
-                            // this loop.  Compact loops: this code runs once per launch
-                            // and straight-line code costs its instruction fetches.
-                            if (lane == 0) RS_TRACE(kRtLnEnter);
-                            float* sc = recv + wk.cr * (N * 32);
-#pragma unroll
-                            for (int t = 0; t < N; ++t) sc[t * 32 + lane] = acc[t];
-                            __syncwarp();
-                            if (lane < N) {
-                                const float* vr = sc + lane * 32;
-                                float m = 0.f;
-#pragma unroll 8
-                                for (int j = 0; j < 32; ++j) m += vr[(j + lane) & 31];
-                                m *= (1.0f / 32.0f);
-                                float q = 0.f;
-#pragma unroll 8
-                                for (int j = 0; j < 32; ++j) {
-                                    const float dv = vr[(j + lane) & 31] - m;
-                                    q = fmaf(dv, dv, q);
-                                }
-                                a.ln_stats[(size_t)lane * (a.RT * 4) + rt * 4 + wk.cr] = make_float2(m, q);
-                            }
-                            // the warp barrier orders every lane's store before lane 0's
-                            // releasing count
-                            __syncwarp();
-                            if (lane == 0) {
-                                red_release_add_gpu(&a.ctl->ln_cnt[par], 1u);
-                                RS_TRACE(kRtLnPublished);
-                            }
-                        }
                     }
-                    // with the LayerNorm, y is stored after its second half
-                    if (ok && a.ln_w == nullptr) {
+                    if (ok) {
                         // rows 32*cr.. of y for all tokens: staged [N tokens][32 rows]
                         // bf16, then one TMA store (rows past T are clipped)
                         if (k > 0 && lane == 0) bulk_wait_group_read0();   // staging free again
@@ -983,7 +903,7 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                             bulk_commit_group();
                             RS_TRACE_ONCE(kRtBReduced);
                         }
-                    } else if (!ok && lane == 0) {
+                    } else if (lane == 0) {
                         sh.b_fail = 1;   // the other warps learn it after the barrier below
                     }
                 }
@@ -998,91 +918,6 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         for (int q = 1; q < kRsCluster; ++q)
                             mbar_arrive_relaxed_cluster(
                                 mapa_shared(smem_u32(&sh.freeB), (uint32_t)((wk.cr + q) % kRsCluster)));
-                    }
-                }
-            }
-        }
-        if (doB && a.ln_w != nullptr && !failed) {
-            // LayerNorm, second half (every row tile of y has its own cluster, so this
-            // block summed one slice, kept in its own receive slot).  All four warps
-            // share the statistics' loads: warp qd takes the quarter qd of the slices
-            // for token `lane` (one round of loads), forms that quarter's mean and M2
-            // (the two-level decomposition, slices in order), and the summing warp
-            // merges the four quarters in order, normalises its 32 rows and stores.
-            named_bar_sync(1, 128);                    // b_fail of the summing warp is final
-            if (et == 0) {
-                int lok = (sh.b_fail == 0 && !sh.abort) ? 1 : 0;
-                if (lok)
-                    lok = wait_count(&a.ctl->ln_cnt[par], (uint32_t)(a.RT * 4), limit_peer, &sh.abort, a.ctl,
-                                     kWaitPeers) ? 1 : 0;
-                sh.ln_ok = lok;
-                RS_TRACE(kRtLnSeen);
-            }
-            named_bar_sync(1, 128);
-            if (sh.ln_ok) {
-                const int nsl = a.RT * 4, nq = nsl / 4;    // slices; per quarter (RT >= 1)
-                float2* part = reinterpret_cast<float2*>(recv + ((wk.cr + 1) & 3) * (N * 32));   // [4][32]
-                {
-                    // nq = RT is even (the single-chunk kernel takes d_h % 256 == 0), so
-                    // a float4 holds two whole slices; 16 slices per batch, their loads
-                    // issued together; two-level within a batch, batches merged in order
-                    // (Chan et al.)
-                    const float4* st4 = reinterpret_cast<const float4*>(a.ln_stats + (size_t)lane * nsl + qd * nq);
-                    float cnt = 0.f, qm = 0.f, qq = 0.f;
-                    for (int j0 = 0; j0 < nq; j0 += 16) {
-                        const int nb = min(16, nq - j0);
-                        float4 v[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            v[u] = 2 * u < nb ? __ldcg(st4 + j0 / 2 + u) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        float sm = 0.f;
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) sm += v[u].x + v[u].z;   // zero past nb
-                        const float bm = sm / (float)nb;
-                        float bq = 0.f;
-#pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            if (2 * u < nb) {
-                                const float d0 = v[u].x - bm, d1 = v[u].z - bm;
-                                bq += v[u].y + 32.f * d0 * d0 + (v[u].w + 32.f * d1 * d1);
-                            }
-                        const float cb = 32.f * (float)nb, ctot = cnt + cb;
-                        const float d = bm - qm;
-                        qm += d * (cb / ctot);
-                        qq += bq + d * d * (cnt * cb / ctot);
-                        cnt = ctot;
-                    }
-                    part[qd * 32 + lane] = make_float2(qm, qq);
-                }
-                named_bar_sync(1, 128);
-                if (qd == wk.cr) {
-                    float mu = 0.f;
-                    for (int w = 0; w < 4; ++w) mu += part[w * 32 + lane].x;
-                    mu *= 0.25f;
-                    float m2 = 0.f;
-                    for (int w = 0; w < 4; ++w) {
-                        const float2 pw = part[w * 32 + lane];
-                        const float d = pw.x - mu;
-                        m2 += pw.y + (32.f * (float)nq) * d * d;
-                    }
-                    const float rstd = 1.0f / sqrtf(m2 / (float)a.d_h + a.ln_eps);
-                    if (lane == 0) RS_TRACE(kRtLnCombined);
-                    const int rt = wk.rt0;                          // the one row tile
-                    const int i = rt * 128 + wk.cr * 32 + lane;     // this lane's row
-                    const float wgt = a.ln_w[i], sft = a.ln_b != nullptr ? a.ln_b[i] : 0.f;
-                    const float* sc = recv + wk.cr * (N * 32);
-#pragma unroll 4
-                    for (int t = 0; t < N; ++t) {
-                        const float mt = __shfl_sync(0xffffffffu, mu, t);
-                        const float rs = __shfl_sync(0xffffffffu, rstd, t);
-                        hstage[t * 32 + lane] = __float2bfloat16_rn(wgt * ((sc[t * 32 + lane] - mt) * rs) + sft);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tm_y, hstage, rt * 128 + wk.cr * 32, 0);
-                        bulk_commit_group();
-                        RS_TRACE_ONCE(kRtBReduced);
                     }
                 }
             }

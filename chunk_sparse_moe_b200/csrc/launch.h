@@ -100,15 +100,8 @@ struct DcArgs {
     __nv_bfloat16* hbuf;      // [E slots][N][d_e] gated activations h'
     uint32_t* readyA;         // [2][E] halves of an expert slot written, by launch parity
     Ctl* ctl;
-    const __nv_bfloat16* x;   // [T, d_h] (the LayerNorm's residual)
     const float* b_in;        // [E, d_e] fc1 biases, or nullptr
     const float* b_out;       // [E, d_h] fc2 biases, or nullptr
-    // LayerNorm(sum + x) in the last step when ln_w != nullptr (every row tile of
-    // y then has a cluster of its own: RT <= clusters); ln_b may be nullptr
-    const float* ln_w;
-    const float* ln_b;
-    float ln_eps;
-    float2* ln_stats;         // [32 tokens][RT*4 slices] (mean, M2) of a 32-row slice
     int T, d_h, E, d_e, n, N;
     int KB;    // d_h / 64
     int RT;    // d_h / 128

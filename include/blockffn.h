@@ -200,10 +200,9 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  * fully overwritten (without LayerNorm, rows of tokens with no active expert are
  * exact zeros).  opts: NULL, or the optional biases and LayerNorm
  * (blockffn_layer_opts); fc2 biases need a workspace sized with
- * BLOCKFFN_WS_EXPERT_BIAS.  The single-chunk kernel applies the LayerNorm in its
- * last step when every row tile of y has a cluster of its own (d_h <= 128 *
- * clusters); otherwise, and on the other paths, a LayerNorm kernel follows the
- * forward on the stream and rewrites y in place.
+ * BLOCKFFN_WS_EXPERT_BIAS.  The LayerNorm is a kernel of its own that follows
+ * the forward on the stream (a programmatic dependent of it) and rewrites y in
+ * place.
  * workspace: ws_bytes >= blockffn_forward_workspace_bytes(...), reset once with
  * blockffn_workspace_reset; it carries state between calls (never share one
  * workspace between calls that may overlap on the GPU).  The first call after a
@@ -217,8 +216,8 @@ blockffn_status blockffn_workspace_reset(void* workspace, size_t ws_bytes, void*
  *   fp32: any d_h, d_e >= 1.
  * Arithmetic: bf16 inputs, fp32 accumulation; the gated Swish activations are
  * rounded to bf16 between the two GEMMs; the biases and the LayerNorm are fp32;
- * y is rounded once to dt (a LayerNorm on the single-chunk kernel works on the
- * fp32 sum; a following LayerNorm kernel reads y as stored).
+ * the expert sum is rounded once to dt, and the LayerNorm reads it as stored and
+ * rounds its result once more.
  * Kernels: one chunk (T <= n, bf16, d_h % 256 == 0) runs the single-chunk
  * cluster kernel; several chunks run the group kernel, which takes whole chunks
  * 256 tokens at a time (128 when T <= 128) and runs each expert of the group's

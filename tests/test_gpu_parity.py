@@ -327,7 +327,8 @@ def test_residual_layernorm_after_the_decode_step(bffn):
     assert_close(out, oracle.residual_layernorm(y_ref, w.x, lg, lb, 1e-5), "bf16", "layer")
 
 
-@pytest.mark.parametrize("T,d_h,dt", [(5, 300, "f32"), (1, 7, "f32"), (33, 2048, "bf16"), (3, 4096, "bf16")])
+@pytest.mark.parametrize("T,d_h,dt", [(5, 300, "f32"), (1, 7, "f32"), (33, 2048, "bf16"), (3, 4096, "bf16"),
+                                      (2, 8200, "bf16"), (3, 12, "bf16"), (2, 5000, "f32")])
 def test_residual_layernorm_shapes(bffn, T, d_h, dt):
     rng = np.random.default_rng(T * 7 + d_h)
     tdt = torch.float32 if dt == "f32" else torch.bfloat16
