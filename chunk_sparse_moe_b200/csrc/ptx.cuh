@@ -183,9 +183,8 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// acquire-release fence at GPU scope (lighter than __threadfence(), whose
-// sequentially consistent fence many blocks issuing at once were measured to
-// serialise: about 0.17 us each, one after another)
+// acquire-release fence at GPU scope: the ordering the release/acquire patterns
+// of these kernels need, without __threadfence()'s sequentially consistent one
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
     uint32_t v;
