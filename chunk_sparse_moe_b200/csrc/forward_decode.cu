@@ -261,8 +261,9 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     const __grid_constant__ CUtensorMap tm_y, const DcArgs a) {
     constexpr int NH = N / 2;   // tokens per k-half block in the expert-in epilogue
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned by pointer arithmetic on the shared array itself (an
+    // integer round trip would make every access through it a generic one)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float* recv = reinterpret_cast<float*>(smem + kRsStages * kRsStageBytes);
     __nv_bfloat16* hstage = reinterpret_cast<__nv_bfloat16*>(smem + kRsStages * kRsStageBytes + kRsRecvBytes);
     RsShared& sh = *reinterpret_cast<RsShared*>(smem + kRsStages * kRsStageBytes + kRsRecvBytes + kRsHStageBytes);

@@ -221,8 +221,9 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     constexpr int kStages = Cfg::kStages;
     constexpr int kStageBytes = Cfg::kStageBytes;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned by pointer arithmetic on the shared array itself (an
+    // integer round trip would make every access through it a generic one)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     GrShared<N>& sh = *reinterpret_cast<GrShared<N>*>(smem + kStages * kStageBytes);
     __nv_bfloat16* ostage = reinterpret_cast<__nv_bfloat16*>(
         (reinterpret_cast<uintptr_t>(&sh + 1) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -595,6 +596,7 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 flush_phase ^= 1u;
                 named_bar_sync(1, kGrEpi);
                 if (!sh.ep_ok) return false;
+                if (et == 0) GR_TRACE(kGtFinBase + 3 * kslot + 1);
 #pragma unroll 1
                 for (int i = et; i < nitems; i += kGrEpi) {
                     const int kq = i / nrows, rr = i - kq * nrows;
@@ -624,7 +626,6 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     }
                 }
                 named_bar_sync(1, kGrEpi);   // the ring is read; the next batch may land
-                if (et == 0) GR_TRACE(kGtFinBase + 3 * kslot + 1);
             }
             if (et == 0) GR_TRACE(kGtFinBase + 3 * kslot + 2);
             return true;
@@ -658,8 +659,15 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 if (npend >= 2) atomicAdd(cntB + pend_sg[1].unit, 1u);
                 GR_TRACE(kGtFlushAnnounced);
             }
-            if (npend >= 1 && !finish_split(pend_sg[0], pend_cb[0], 0)) return false;
-            if (npend >= 2 && !finish_split(pend_sg[1], pend_cb[1], 1)) return false;
+            // one copy of the finisher's code, run once per pending unit (its
+            // instructions are fetched cold once per launch, not once per call
+            // site); the slot is picked field by field, in registers
+#pragma unroll 1
+            for (int k = 0; k < npend; ++k) {
+                const GrSeg sgk = k == 0 ? pend_sg[0] : pend_sg[1];
+                const GrContrib cbk = k == 0 ? pend_cb[0] : pend_cb[1];
+                if (!finish_split(sgk, cbk, k)) return false;
+            }
             npend = 0;
             return true;
         };
