@@ -570,8 +570,11 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             }
             named_bar_sync(1, kGrEpi);
             if (!sh.ep_ok) return false;
-            const int r0 = cb.rank * 128 / cb.n, r1 = (cb.rank + 1) * 128 / cb.n;
-            const int nrows = r1 - r0;                        // <= 64
+            // rows in whole 8-row pieces (16-byte stores of y): rank r of n takes
+            // [8 floor(16 r / n), 8 floor(16 (r + 1) / n)), possibly none
+            const int r0 = 8 * (cb.rank * 16 / cb.n), r1 = 8 * ((cb.rank + 1) * 16 / cb.n);
+            const int nrows = r1 - r0;                        // <= 64 (n >= 2), a multiple of 8
+            if (nrows == 0) return true;                      // (the same in every thread)
             const int nb = (nrows + 31) / 32;                 // boxes per contributor
             const int cap = kRingBoxes / nb - 1;              // contributors per batch
             const int nitems = nrows * (N / 4);               // (row, token quad) items
@@ -597,35 +600,69 @@ union_expert_group(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 named_bar_sync(1, kGrEpi);
                 if (!sh.ep_ok) return false;
                 if (et == 0) GR_TRACE(kGtFinBase + 3 * kslot + 1);
+                if (!last) {
+                    // running sums of this batch's contributors
 #pragma unroll 1
-                for (int i = et; i < nitems; i += kGrEpi) {
-                    const int kq = i / nrows, rr = i - kq * nrows;
-                    const int off = (rr >> 5) * kBoxF4 + kq * 32 + (rr & 31);
-                    float4 acc = c0 == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ring4[off];
+                    for (int i = et; i < nitems; i += kGrEpi) {
+                        const int kq = i / nrows, rr = i - kq * nrows;
+                        const int off = (rr >> 5) * kBoxF4 + kq * 32 + (rr & 31);
+                        float4 acc = c0 == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ring4[off];
 #pragma unroll 1
-                    for (int c = 0; c < cn; ++c) {
-                        const float4 v = ring4[(1 + c) * nb * kBoxF4 + off];
-                        acc.x += v.x;
-                        acc.y += v.y;
-                        acc.z += v.z;
-                        acc.w += v.w;
-                    }
-                    if (!last) {
+                        for (int c = 0; c < cn; ++c) {
+                            const float4 v = ring4[(1 + c) * nb * kBoxF4 + off];
+                            acc.x += v.x;
+                            acc.y += v.y;
+                            acc.z += v.z;
+                            acc.w += v.w;
+                        }
                         ring4[off] = acc;
-                    } else {
-                        const size_t col = (size_t)sg.g * a.NT * a.d_h + sg.rt * 128 + r0 + rr;
-                        __nv_bfloat16* ycol = a.y + col;
+                    }
+                    named_bar_sync(1, kGrEpi);   // the ring is read; the next batch may land
+                    continue;
+                }
+                // the last batch: 128 tokens at a time, the sums (plus the fc2 bias
+                // sums) rounded into the output staging [128 tokens][64 rows], then
+                // written as 16-byte pieces of 8 rows
+#pragma unroll 1
+                for (int h = 0; h < N / 128; ++h) {
+#pragma unroll 1
+                    for (int i = et; i < nrows * 32; i += kGrEpi) {
+                        const int kql = i / nrows, rr = i - kql * nrows;
+                        const int kq = 32 * h + kql;
+                        const int off = (rr >> 5) * kBoxF4 + kq * 32 + (rr & 31);
+                        float4 acc = c0 == 0 ? make_float4(0.f, 0.f, 0.f, 0.f) : ring4[off];
+#pragma unroll 1
+                        for (int c = 0; c < cn; ++c) {
+                            const float4 v = ring4[(1 + c) * nb * kBoxF4 + off];
+                            acc.x += v.x;
+                            acc.y += v.y;
+                            acc.z += v.z;
+                            acc.w += v.w;
+                        }
                         const float z[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            if (4 * kq + u < nvalid) {
-                                const size_t o = (size_t)(4 * kq + u) * a.d_h;
-                                const float yb = a.ybias != nullptr ? __ldg(a.ybias + col + o) : 0.f;
-                                ycol[o] = __float2bfloat16_rn(z[u] + yb);
-                            }
+                        for (int u = 0; u < 4; ++u) {
+                            const int tok = 4 * kq + u;
+                            const float yb = (a.ybias != nullptr && tok < nvalid)
+                                                 ? __ldg(a.ybias + (size_t)(sg.g * a.NT + tok) * a.d_h + sg.rt * 128 +
+                                                         r0 + rr)
+                                                 : 0.f;
+                            ostage[(4 * kql + u) * 64 + rr] = __float2bfloat16_rn(z[u] + yb);
+                        }
                     }
+                    named_bar_sync(1, kGrEpi);
+                    const int np = nrows / 8;
+#pragma unroll 1
+                    for (int c = et; c < 128 * np; c += kGrEpi) {
+                        const int tl = c / np, pc = c - tl * np;
+                        const int tok = 128 * h + tl;
+                        if (tok < nvalid)
+                            *reinterpret_cast<uint4*>(a.y + (size_t)(sg.g * a.NT + tok) * a.d_h + sg.rt * 128 + r0 +
+                                                      8 * pc) =
+                                *reinterpret_cast<const uint4*>(ostage + tl * 64 + 8 * pc);
+                    }
+                    named_bar_sync(1, kGrEpi);   // the staging and the ring are free again
                 }
-                named_bar_sync(1, kGrEpi);   // the ring is read; the next batch may land
             }
             if (et == 0) GR_TRACE(kGtFinBase + 3 * kslot + 2);
             return true;
