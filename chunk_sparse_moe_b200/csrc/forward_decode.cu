@@ -44,7 +44,8 @@
 //
 // Roles (224 threads): warp 0 TMA producer (one lane), warp 1 MMA issuer (the
 // whole warp runs its loops and waits, one elected lane issues), warp 2 TMEM
-// owner and h' loader, warps 3-6 epilogue.  Every wait is bounded; a timeout
+// owner and activation loader (x; the even expert-out stages' h'), warps 3-6
+// epilogue (one lane of warp 6, or 5, also issues the odd stages' h' copies).  Every wait is bounded; a timeout
 // records BLOCKFFN_ERR_TIMEOUT and the block winds down without leaving copies
 // in flight.
 //
@@ -599,15 +600,20 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
         }
         stop = __shfl_sync(0xffffffffu, stop, 0);
+        const long long iB0 = i;   // ring index of the first expert-out stage
         if (!stop && totB > 0 && lane == 0) {
             // Each expert-out tile waits (bounded) only for its own expert slot's h'
             // (both k-halves of every 128-row tile counted in), so tiles of experts
             // finished early start while later experts' expert-in units still run.
+            // This thread takes the even tiles; an epilogue lane (warp 6, or 5 in
+            // rank 2) issues the odd ones (one thread issues bulk copies at a bounded
+            // rate, and the expert-out phase is one h' copy per stage).
             const uint64_t pol = policy_evict_first();
             BCursor bc;
             bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
             int ready_s = -1;
             for (int q = 0; q < totB; ++q, ++i, rp.advance(), bc.advance()) {
+                if (q & 1) continue;
                 if (bc.s != ready_s) {
                     if (!wait_count(&readyA[bc.s], (uint32_t)(2 * MT), limit_peer, &sh.abort, a.ctl)) break;
                     // the h' stores were made visible to this thread by the acquire;
@@ -627,9 +633,11 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         if (lane == 0) {
             // no copy into this block's shared memory outlives it: the last ring's
             // worth of stages this warp filled (x or h'; an earlier stage's slot was
-            // only refilled after the MMAs had read it, so its copy had landed)
+            // only refilled after the MMAs had read it, so its copy had landed); the
+            // odd expert-out stages are the epilogue lane's, which drains its own
             for (long long q = i - kRsStages < 0 ? 0 : i - kRsStages; q < i; ++q)
-                wait_bar_drain(&sh.full_h[q % kRsStages], (uint32_t)((q / kRsStages) & 1), limit, a.ctl);
+                if (q < iB0 || ((q - iB0) & 1) == 0)
+                    wait_bar_drain(&sh.full_h[q % kRsStages], (uint32_t)((q / kRsStages) & 1), limit, a.ctl);
         }
     } else {
         // --------------------------------------------------------- epilogue --
@@ -783,6 +791,48 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         }
         named_bar_sync(1, 128);
         failed = failed || !sh.b_go;
+        // one lane of a warp that is neither the summing warp of this rank (whose
+        // fc2 bias sums overlap the MMAs) nor warp 3 (whose lane 0 takes the
+        // epilogue's waits)
+        if (warp == (wk.cr == 2 ? 5 : 6) && lane == 0 && !failed && totB > 0) {
+            // The odd expert-out stages' h' copies (the loader issues the even ones):
+            // the same per-expert readiness wait, then one TMA copy into the stage.
+            // This lane then drains its own copies that may still be in flight: its
+            // stages among the last ring's worth of all expert-out stages (an earlier
+            // slot was refilled by a later stage, issued only after the MMAs had read
+            // it, so its copy had landed; and no stage follows the last ones, so the
+            // parity of their phase is not ambiguous), before rejoining the
+            // epilogue's barriers.
+            const uint64_t pol = policy_evict_first();
+            long long ib = (long long)wk.nA * KP;
+            RingPos bp;
+            bp.st = (int)(ib % kRsStages);
+            bp.ph = (uint32_t)((ib / kRsStages) & 1);
+            BCursor bc;
+            bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
+            int ready_s = -1;
+            long long last = -1;
+            int q = 0;
+            for (; q < totB; ++q, ++ib, bp.advance(), bc.advance()) {
+                if ((q & 1) == 0) continue;
+                if (bc.s != ready_s) {
+                    if (!wait_count(&readyA[bc.s], (uint32_t)(2 * MT), limit_peer, &sh.abort, a.ctl)) break;
+                    fence_proxy_async_global();
+                    ready_s = bc.s;
+                }
+                if (!wait_bar(&sh.empty[bp.st], bp.ph ^ 1u, limit, &sh.abort, a.ctl, kWaitEmpty)) break;
+                mbar_arrive_expect_tx(&sh.full_h[bp.st], (uint32_t)(N * 256));
+                tma_load_3d(smem + bp.st * kRsStageBytes + kRsWBytes, &tm_h, &sh.full_h[bp.st], 0, bc.s * N,
+                            2 * bc.kb, pol);
+                last = ib;
+            }
+            // (after an early exit, the window ends at this lane's last stage)
+            const long long ib0 = (long long)wk.nA * KP, iend = q == totB ? ib0 + totB : last + 1;
+            for (long long q2 = iend - kRsStages < ib0 ? ib0 : iend - kRsStages; q2 <= last; ++q2)
+                if (((q2 - ib0) & 1) == 1)
+                    wait_bar_drain(&sh.full_h[q2 % kRsStages], (uint32_t)((q2 / kRsStages) & 1), limit, a.ctl);
+        }
+        __syncwarp();
         if (doB) {
             const uint32_t recv_u32 = smem_u32(recv);
             for (int k = 0; k < wk.nRT && !failed; ++k) {
