@@ -224,37 +224,6 @@ __device__ __forceinline__ RsWork rs_work(int G, int P, int MT, int KPe, int RT)
     return w;
 }
 
-// Sums over the warp's 32 lanes of one value per token, scattered: on return
-// lane j holds the sum over the lanes of v[j % N] (v is consumed).  A fixed
-// butterfly, so the sums do not depend on timing.
-template <int N>
-__device__ __forceinline__ float rs_warp_sum_scatter(float (&v)[N]) {
-    const int lane = threadIdx.x & 31;
-    if constexpr (N == 16) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 16);
-    }
-#pragma unroll
-    for (int off = N / 2; off >= 1; off >>= 1) {
-        const bool up = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < off; ++i) {
-            const float send = up ? v[i] : v[i + off];
-            const float keep = up ? v[i + off] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-    }
-    return v[0];
-}
-
-// The same total in every lane (an xor butterfly: every lane adds the same two
-// values at every level, so all lanes hold the same bits).
-__device__ __forceinline__ float rs_warp_allsum(float v) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
-}
-
 template <int N>
 __global__ void __launch_bounds__(kRsThreads, 1)
 union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_win,

@@ -309,7 +309,8 @@ void blockffn_debug_skip_flag(int unit);
  * slice staged; for the first unit's slices s = 0..7, 16 + 4s + {0: TMEM read,
  * 1: staged, 2: barrier passed, 3: stores issued}; 48 expert-out partials
  * written, 49 announced, and for pending split unit k = 0, 1: 50 + 3k
- * contributors counted, 51 + 3k partials summed, 52 + 3k rows of y stored.
+ * contributors counted, 51 + 3k first batch of partials landed, 52 + 3k rows of
+ * y stored.
  * Single-chunk launches: 0 start, 1 prologue done,
  * 2 first weight load issued, 3 last load issued, 4 first expert-in tile landed,
  * 5 last expert-in accumulator committed, 7 expert-in units finished, 8 first and
@@ -317,7 +318,8 @@ void blockffn_debug_skip_flag(int unit);
  * committed, 11 last epilogue step, 13 end; for the block's first expert-in unit:
  * 14 accumulator read, 15 partial sent to the peer, 16 peer's partial received,
  * 17 peer's partial read, 18 h' published; 21 first expert-out quadrant sent,
- * 23 first 32 rows of y summed and stored, 24 first expert-out MMA issued.
+ * 23 first 32 rows of y summed and stored, 24 first expert-out MMA issued,
+ * 30 the other ranks' expert-out partials received (summing warp).
  * Unset stamps stay 0.  NULL (the default) turns tracing off.
  */
 void blockffn_debug_set_trace(void* device_buffer);
