@@ -279,6 +279,22 @@ def test_deterministic_and_workspace_reuse(bffn):
     assert bffn.device_status(ws) == (0, 0)
 
 
+def test_repeated_calls_alternating_inputs(bffn):
+    """Many single-chunk launches on fresh and reused workspaces, two inputs in
+    turn: every output matches the oracle and no launch records an error.  (A
+    barrier-phase mistake in the expert-out copies showed up here as an
+    intermittent timeout, in about one trial of three, never in one call.)"""
+    w = wl.chunk32()
+    w2 = wl.chunk32(weights=(w.W_in, w.W_out), x_seed=77)
+    refs = {id(w): oracle_y(w, w.gates.astype(np.float64)), id(w2): oracle_y(w2, w2.gates.astype(np.float64))}
+    for trial in range(12):
+        ws = bffn.Workspace.for_shapes(w.T, w.d_h, w.E, w.d_e, w.n, torch.bfloat16, False)
+        for k, ww in enumerate((w, w2, w2, w, w2)):
+            y, _ = run_gpu(ww, ws)
+            assert_close(y, refs[id(ww)], "bf16", f"trial {trial} call {k}")
+        assert bffn.device_status(ws) == (0, 0)
+
+
 def test_chained_launches_read_the_previous_output(bffn):
     """Each forward's input is the previous forward's output, launched back to back
     on one stream with no host synchronisation: the single-chunk kernel may begin
