@@ -14,10 +14,13 @@ events around each launch give the kernel's own time for the roofline.
 
 The JSON line also carries: the end-to-end number through the public API with
 host buffers (x and gates copied in from pinned memory, y copied out, every
-step), the same-size dense FFN on the GPU (torch bf16 matmuls) and the routed
-decode step (router + forward) for context, the HBM roofline fraction on
-union-expert bytes, the fp64 CPU oracle timed on a bounded sample (rank 0, one
-GPU), and the SM clocks sampled during the run.
+step), the same-size dense FFN on the GPU (torch bf16 matmuls), the routed
+decode step (router + forward) and the step with the layer's optional expert
+biases and LayerNorm for context, the HBM roofline fraction on union-expert
+bytes, the fp64 CPU oracle timed on a bounded sample (rank 0, one GPU), the SM
+clocks sampled during the run, and the other workloads (batch16, seq4096 and
+the d_h 4096 sweep, each beside its dense FFN; ``--workloads`` /
+``--no-workloads``).
 
 ``--impl reference`` times the fp64 CPU oracle alone on the same workload and
 metric: the pages ship no runnable implementation of the layer, so the oracle
