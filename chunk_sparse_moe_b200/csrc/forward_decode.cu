@@ -45,7 +45,8 @@
 // Roles (224 threads): warp 0 TMA producer (one lane), warp 1 MMA issuer (the
 // whole warp runs its loops and waits, one elected lane issues), warp 2 TMEM
 // owner and activation loader (x; the even expert-out stages' h'), warps 3-6
-// epilogue (one lane of warp 6, or 5, also issues the odd stages' h' copies).  Every wait is bounded; a timeout
+// epilogue (one lane of warp 6, or 5, also issues the odd expert-out stages' h'
+// copies of the first two row tiles).  Every wait is bounded; a timeout
 // records BLOCKFFN_ERR_TIMEOUT and the block winds down without leaving copies
 // in flight.
 //
@@ -110,6 +111,8 @@ struct RsShared {
     int P;
     uint32_t trace_once;          // trace slots already stamped (first occurrence only)
     int pendA[2], pendB;          // parity of a receive phase armed but not seen complete, or -1
+    long long h_last;             // ring index of the last h' copy the epilogue lane issued, or -1
+    int mma_all;                  // the MMAs read every stage of the launch (so every copy landed)
     float s_gate[2][32];          // gates of the current expert-in unit's expert, per token
     int32_t s_pair_e[kRsMaxE];    // the union, ascending
     uint32_t s_tmask[kRsMaxE];    // per expert: bit t = token t's gate is nonzero
@@ -265,6 +268,8 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         mbar_init(&sh.a_pub, 1);
         sh.trace_once = 0u;
         sh.pendA[0] = sh.pendA[1] = sh.pendB = -1;
+        sh.h_last = -1;
+        sh.mma_all = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_x);
         prefetch_tmap(&tm_win);
@@ -366,6 +371,13 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     const int nBt = wk.bHi - wk.bLo;                 // expert-out tiles per owned row tile
     const int totB = P > 0 ? wk.nRT * nBt : 0;        // this block's expert-out tiles
     const bool doB = P > 0 && wk.nRT > 0;             // this cluster sums expert-out row tiles
+    // The expert-out stages' h' copies of the first two row tiles alternate
+    // between the loader (even) and one epilogue lane (odd); later row tiles are
+    // the loader's alone (their MMAs wait for an accumulator the epilogue frees,
+    // which that lane, held at the epilogue's barrier, could not wait for).
+    const int qsplit = min(totB, 2 * nBt);
+    const long long iB0 = (long long)wk.nA * (a.KB / 4);   // ring index of the first expert-out stage
+    long long ld_last = -1;                           // the loader's last issued ring index
     if (threadIdx.x == 0 && doB && !sh.abort) {
         // the first expert-out reduction: 3 quadrant partials of 32 rows x N tokens
         // (not armed by a launch that computes nothing, whose teardown would
@@ -540,7 +552,11 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
             __syncwarp();
         }
-        if (leader) umma_commit(&sh.mma_done);
+        if (leader) {
+            // every stage read: each copy issued into the ring has landed
+            if (i == (long long)wk.nA * KP + totB) sh.mma_all = 1;
+            umma_commit(&sh.mma_done);
+        }
         __syncwarp();
     } else if (warp == 2) {
         // ------------------------------------------------- activation loader --
@@ -565,24 +581,25 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 256));
                     tma_load_3d(smem + rp.st * kRsStageBytes + kRsWBytes, &tm_x, &sh.full_h[rp.st], 0, 0,
                                 2 * (wk.hk * KP + t), pol_keep);
+                    ld_last = i;
                 }
             }
         }
         stop = __shfl_sync(0xffffffffu, stop, 0);
-        const long long iB0 = i;   // ring index of the first expert-out stage
         if (!stop && totB > 0 && lane == 0) {
             // Each expert-out tile waits (bounded) only for its own expert slot's h'
             // (both k-halves of every 128-row tile counted in), so tiles of experts
             // finished early start while later experts' expert-in units still run.
-            // This thread takes the even tiles; an epilogue lane (warp 6, or 5 in
-            // rank 2) issues the odd ones (one thread issues bulk copies at a bounded
-            // rate, and the expert-out phase is one h' copy per stage).
+            // Of the first two row tiles this thread takes the even stages and an
+            // epilogue lane (warp 6, or 5 in rank 2) the odd ones (one thread issues
+            // bulk copies at a bounded rate, and the expert-out phase is one h'
+            // copy per stage); later row tiles' stages are all this thread's.
             const uint64_t pol = policy_evict_first();
             BCursor bc;
             bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
             int ready_s = -1;
             for (int q = 0; q < totB; ++q, ++i, rp.advance(), bc.advance()) {
-                if (q & 1) continue;
+                if (q < qsplit && (q & 1)) continue;
                 if (bc.s != ready_s) {
                     if (!wait_count(&readyA[bc.s], (uint32_t)(2 * MT), limit_peer, &sh.abort, a.ctl)) break;
                     // the h' stores were made visible to this thread by the acquire;
@@ -596,18 +613,11 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 mbar_arrive_expect_tx(&sh.full_h[rp.st], (uint32_t)(N * 256));
                 tma_load_3d(smem + rp.st * kRsStageBytes + kRsWBytes, &tm_h, &sh.full_h[rp.st], 0, bc.s * N,
                             2 * bc.kb, pol);
+                ld_last = i;
             }
         }
         __syncwarp();
-        if (lane == 0) {
-            // no copy into this block's shared memory outlives it: the last ring's
-            // worth of stages this warp filled (x or h'; an earlier stage's slot was
-            // only refilled after the MMAs had read it, so its copy had landed); the
-            // odd expert-out stages are the epilogue lane's, which drains its own
-            for (long long q = i - kRsStages < 0 ? 0 : i - kRsStages; q < i; ++q)
-                if (q < iB0 || ((q - iB0) & 1) == 0)
-                    wait_bar_drain(&sh.full_h[q % kRsStages], (uint32_t)((q / kRsStages) & 1), limit, a.ctl);
-        }
+        // (this warp's copies are drained at teardown, with the epilogue lane's)
     } else {
         // --------------------------------------------------------- epilogue --
         cluster_wait_acquire();
@@ -763,26 +773,20 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         // one lane of a warp that is neither the summing warp of this rank (whose
         // fc2 bias sums overlap the MMAs) nor warp 3 (whose lane 0 takes the
         // epilogue's waits)
-        if (warp == (wk.cr == 2 ? 5 : 6) && lane == 0 && !failed && totB > 0) {
-            // The odd expert-out stages' h' copies (the loader issues the even ones):
-            // the same per-expert readiness wait, then one TMA copy into the stage.
-            // This lane then drains its own copies that may still be in flight: its
-            // stages among the last ring's worth of all expert-out stages (an earlier
-            // slot was refilled by a later stage, issued only after the MMAs had read
-            // it, so its copy had landed; and no stage follows the last ones, so the
-            // parity of their phase is not ambiguous), before rejoining the
-            // epilogue's barriers.
+        if (warp == (wk.cr == 2 ? 5 : 6) && lane == 0 && !failed && qsplit > 1) {
+            // The odd expert-out stages' h' copies of the first two row tiles (the
+            // loader issues the rest): the same per-expert readiness wait, then one
+            // TMA copy into the stage; the last ring index issued goes to shared
+            // memory for the teardown's drain.
             const uint64_t pol = policy_evict_first();
-            long long ib = (long long)wk.nA * KP;
+            long long ib = iB0;
             RingPos bp;
             bp.st = (int)(ib % kRsStages);
             bp.ph = (uint32_t)((ib / kRsStages) & 1);
             BCursor bc;
             bc.init(wk.rt0, wk.rtstep, wk.bLo, wk.bHi, KPe);
             int ready_s = -1;
-            long long last = -1;
-            int q = 0;
-            for (; q < totB; ++q, ++ib, bp.advance(), bc.advance()) {
+            for (int q = 0; q < qsplit; ++q, ++ib, bp.advance(), bc.advance()) {
                 if ((q & 1) == 0) continue;
                 if (bc.s != ready_s) {
                     if (!wait_count(&readyA[bc.s], (uint32_t)(2 * MT), limit_peer, &sh.abort, a.ctl)) break;
@@ -793,13 +797,8 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 mbar_arrive_expect_tx(&sh.full_h[bp.st], (uint32_t)(N * 256));
                 tma_load_3d(smem + bp.st * kRsStageBytes + kRsWBytes, &tm_h, &sh.full_h[bp.st], 0, bc.s * N,
                             2 * bc.kb, pol);
-                last = ib;
+                sh.h_last = ib;
             }
-            // (after an early exit, the window ends at this lane's last stage)
-            const long long ib0 = (long long)wk.nA * KP, iend = q == totB ? ib0 + totB : last + 1;
-            for (long long q2 = iend - kRsStages < ib0 ? ib0 : iend - kRsStages; q2 <= last; ++q2)
-                if (((q2 - ib0) & 1) == 1)
-                    wait_bar_drain(&sh.full_h[q2 % kRsStages], (uint32_t)((q2 / kRsStages) & 1), limit, a.ctl);
         }
         __syncwarp();
         if (doB) {
@@ -957,6 +956,28 @@ union_expert_decode(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         if (sh.pendB >= 0) wait_bar_drain(&sh.recvB, (uint32_t)sh.pendB, limit, a.ctl);
     }
     if (warp == 2) {
+        if (lane == 0 && !sh.mma_all) {
+            // No activation copy into this block's shared memory outlives it.  When
+            // the MMAs read every stage, every copy landed; otherwise (a launch that
+            // gave up), for every ring slot the last copy issued into it (by the
+            // loader or the epilogue lane) is waited for: an earlier copy into a slot
+            // was followed by a later one, issued only after the MMAs had read the
+            // slot, so it had landed; and no copy followed the last one, so the
+            // parity of its phase is not ambiguous.
+            const long long h_last = sh.h_last;
+            const long long last = ld_last > h_last ? ld_last : h_last;
+            int found = 0;
+            for (long long pos = last; pos >= 0 && found != (1 << kRsStages) - 1; --pos) {
+                const int slot = (int)(pos % kRsStages);
+                if (found & (1 << slot)) continue;
+                const long long qb = pos - iB0;   // expert-out stage, or negative: expert-in
+                const bool helper = qb >= 0 && qb < qsplit && (qb & 1);
+                if (helper ? pos <= h_last : pos <= ld_last) {
+                    found |= 1 << slot;
+                    wait_bar_drain(&sh.full_h[slot], (uint32_t)((pos / kRsStages) & 1), limit, a.ctl);
+                }
+            }
+        }
         if (lane == 0) wait_bar_drain(&sh.mma_done, 0, limit, a.ctl);
         __syncwarp();
         tc_fence_after();

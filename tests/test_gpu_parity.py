@@ -130,6 +130,7 @@ def test_forward_tiny_f32_router(bffn):
     (96, 32, 1024, 64, 128, "markov90"),
     (40, 17, 256, 32, 384, "markov80"),    # d_e = 384, n = 17 (N = 32)
     (32, 32, 8192, 16, 128, "markov80"),   # one chunk, 64 row tiles: clusters own two each
+    (32, 32, 16384, 8, 128, "all_on"),     # one chunk, 128 row tiles: clusters own four each
 ])
 def test_forward_bf16_small(bffn, T, n, d_h, E, d_e, regime):
     w = wl.make_injected("small", T, n, d_h, E, d_e, "bf16", regime, seed=T + d_h + E)
