@@ -287,7 +287,7 @@ def measure_workloads(dev, stream, with_oracle: bool, which=("batch16", "seq4096
     if "seq4096" in which:
         out["seq4096"] = _seq4096(dev, stream, d, dense_us, with_oracle)
     if "sweep" in which:
-        out["sweep"] = _sweep(dev, stream, d, dense_us)
+        out["sweep"] = _sweep(dev, stream, d, dense_us, with_oracle)
     return out
 
 
@@ -369,7 +369,7 @@ def _seq4096(dev, stream, d, dense_us, with_oracle):
     return out
 
 
-def _sweep(dev, stream, d, dense_us):
+def _sweep(dev, stream, d, dense_us, with_oracle=False):
     """d_h 4096, E 128: every chunk of the 4096-token sequence as its own decode
     call, n in {1, 8, 32}, four gate regimes (256 MiB of weights > L2)."""
     import torch
@@ -403,10 +403,14 @@ def _sweep(dev, stream, d, dense_us):
                          "dense_ffn_us": dense_cache[n],
                          "speedup_vs_dense": dense_cache[n] / us})
         del ws
-    return {"what": "d_h 4096, E 128, d_e 128, bf16, T 4096: every chunk of the sequence as its own decode "
-                    "call (a graph of the consecutive calls), mean per call; dense = the same-size dense FFN "
-                    "on n tokens (torch bf16)",
-            "rows": rows}
+    out = {"what": "d_h 4096, E 128, d_e 128, bf16, T 4096: every chunk of the sequence as its own decode "
+                   "call (a graph of the consecutive calls), mean per call; dense = the same-size dense FFN "
+                   "on n tokens (torch bf16)",
+           "rows": rows}
+    if with_oracle:
+        # the dense fp64 definition costs the same in every regime: one 32-token chunk
+        out["cpu_baseline"] = oracle_sample(wl.sweep(32, "markov80"), 32, False)
+    return out
 
 
 def run_reference(args, world, rank):
