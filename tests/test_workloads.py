@@ -115,3 +115,21 @@ def test_accept_lengths_match_their_closed_form():
         assert abs(a.mean() - m) <= 4.0 * sd / np.sqrt(a.size) + 1e-12, (n, p, a.mean(), m)
     assert np.all(wl.accept_lengths(0, 10, 32, 0.0) == 1)
     assert np.all(wl.accept_lengths(0, 10, 32, 1.0) == 33)
+
+
+def test_expert_biases_and_layernorm_params():
+    """Bias generators: nn.Linear's initial U(-1/sqrt(fan_in), 1/sqrt(fan_in)) times
+    the scale, fp32, seeded; LayerNorm scale in [0.5, 1.5], small shifts."""
+    E, d_e, d_h = 6, 128, 512
+    b_in, b_out = wl.expert_biases(3, E, d_e, d_h)
+    assert b_in.shape == (E, d_e) and b_out.shape == (E, d_h)
+    assert b_in.dtype == np.float32 and b_out.dtype == np.float32
+    assert np.max(np.abs(b_in)) <= 1.0 / np.sqrt(d_h) and np.max(np.abs(b_out)) <= 1.0 / np.sqrt(d_e)
+    # uniform: the spread fills most of the interval
+    assert np.max(b_out) > 0.9 / np.sqrt(d_e) and np.min(b_out) < -0.9 / np.sqrt(d_e)
+    b_in2, b_out2 = wl.expert_biases(3, E, d_e, d_h, scale=4.0)
+    assert np.allclose(b_in2, 4.0 * b_in) and np.allclose(b_out2, 4.0 * b_out)
+    assert np.array_equal(wl.expert_biases(3, E, d_e, d_h)[0], b_in)
+    lw, lb = wl.layernorm_params(5, d_h)
+    assert lw.shape == lb.shape == (d_h,) and lw.dtype == lb.dtype == np.float32
+    assert np.all((lw >= 0.5) & (lw <= 1.5)) and abs(float(np.std(lb)) - 0.1) < 0.02
